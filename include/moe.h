@@ -1,0 +1,167 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) Grok-1 MoE feed-forward sublayer.
+ *
+ * The operation (grok-field-guide "Grok-1 blueprint", section "MoE sublayer";
+ * Grok-1 book ch. 10 "Comparison with other MoE", sections 10.3, 10.3.1, 10.4):
+ *   for every token t (row of x):
+ *     logits = x[t] . w_router (+ router_bias)           fp32, 8 experts
+ *     p      = softmax(logits)                           fp32
+ *     (e0,e1)= the two largest logits, descending; an exact tie goes to the
+ *              lower expert index; gates g0 = p[e0], g1 = p[e1], NOT renormalised
+ *     y_s    = ( GELU(x[t] . w_gate[e_s]) * (x[t] . w_up[e_s]) ) . w_down[e_s]
+ *     out[t] = g0 * y_0 + g1 * y_1
+ *   GELU is the tanh approximation unless MOE_GELU_ERF is asked for. Every
+ *   routed (token, expert) pair is computed: no capacity limit, no token drop
+ *   (Grok-1 book ch. 10, section 10.3.2, capacity-factor box).
+ *
+ * Pointers. Every array argument is a DEVICE pointer on the device that owns
+ * `stream`; the caller owns all of them; the library never frees or retains
+ * them and never synchronises the stream. All arrays are dense, row-major,
+ * 16-byte aligned:
+ *   x        [T, d]      fp32 (MOE_F32) or bf16 (MOE_BF16, MOE_BF16_INT8W)
+ *   w_router [d, E]      fp32 (always)
+ *   w_gate   [E, d, f]   fp32 / bf16 / int8 (by dtype)
+ *   w_up     [E, d, f]   fp32 / bf16 / int8
+ *   w_down   [E, f, d]   fp32 / bf16 / int8
+ *   out      [T, d]      same dtype as x
+ * int8 weights carry one bf16 scale per output channel (Grok-1 book ch. 1,
+ * section 1.2, INT8 box): w = q * s, s_gate/s_up [E, f], s_down [E, d].
+ *
+ * Limits of this version: E == 8, k == 2; MOE_F32 needs d % 64 == 0 and
+ * f % 64 == 0; MOE_BF16 and MOE_BF16_INT8W need d % 256 == 0 and f % 128 == 0;
+ * 0 <= T <= 2^24. T == 0 returns MOE_OK and launches nothing.
+ *
+ * Errors. Arguments are checked on the host before anything is launched; a
+ * failed check returns its status and launches nothing. A launch failure
+ * returns MOE_ERR_CUDA. Faults of earlier asynchronous work surface at the
+ * caller's next synchronisation, not here. Kernels never trap: a wait that
+ * exceeds its time limit records a code in the workspace status word, which
+ * moe_device_status() reads back as MOE_ERR_DEVICE_CHECK. Behaviour on
+ * non-finite inputs is unspecified.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_EXPORT __attribute__((visibility("default")))
+#else
+#define MOE_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size   */
+  MOE_ERR_UNSUPPORTED = 2,   /* E != 8, k != 2, or d / f not a supported multiple */
+  MOE_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned              */
+  MOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than needed      */
+  MOE_ERR_CUDA = 5,          /* a CUDA runtime / driver call failed           */
+  MOE_ERR_DEVICE_CHECK = 6   /* a kernel recorded a device-side check failure */
+} moe_status_t;
+
+typedef enum {
+  MOE_F32 = 0,         /* fp32 activations and weights, fp32 arithmetic        */
+  MOE_BF16 = 1,        /* bf16 activations and weights, fp32 accumulation      */
+  MOE_BF16_INT8W = 2   /* bf16 activations, int8 weights + bf16 channel scales */
+} moe_dtype_t;
+
+typedef enum { MOE_GELU_TANH = 0, MOE_GELU_ERF = 1 } moe_gelu_t;
+
+/* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
+ * down projection) when the average tokens per expert is small, else
+ * TOKEN_TILE (128-token tiles on the MMA M side). Both compute the same result. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_TOKEN_TILE = 1, MOE_PATH_WEIGHT_STREAM = 2 } moe_path_t;
+
+/* Per-output-channel scales of int8 weights (device pointers, bf16). */
+typedef struct {
+  const void* s_gate; /* [E, f] */
+  const void* s_up;   /* [E, f] */
+  const void* s_down; /* [E, d] */
+} moe_scales_t;
+
+/* cudaStream_t, passed as an opaque handle (NULL = the legacy default stream). */
+typedef void* moe_stream_t;
+
+/* All arguments of one forward call (see the file header for layouts). */
+typedef struct {
+  const void* x;
+  const float* w_router;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+  const moe_scales_t* w_scales; /* host struct of device pointers; NULL unless MOE_BF16_INT8W */
+  void* out;
+  int64_t T, d, f;
+  int32_t E, k;
+  moe_dtype_t dtype;
+} moe_args_t;
+
+typedef struct {
+  moe_gelu_t gelu;            /* MOE_GELU_TANH (default) or MOE_GELU_ERF             */
+  const float* router_bias;   /* [E] fp32 device pointer added to the logits, or NULL */
+  moe_path_t path;            /* kernel family; MOE_PATH_AUTO by default             */
+  int32_t down_splits;        /* WEIGHT_STREAM split-K factor for w_down; 0 = auto    */
+  void* const* stage_events;  /* NULL, or 6 cudaEvent_t (host array) recorded on the
+                                 stream before router, dispatch, gate/up GEMM, down
+                                 GEMM, combine, and after combine (stage timing)     */
+} moe_options_t;
+
+/* Optional outputs for inspection; each is a device pointer or NULL.
+ * Permuted order = token slots sorted stably by (expert, token). */
+typedef struct {
+  int32_t* idx;        /* [T, 2] chosen experts, slot 0 = larger logit      */
+  float* gates;        /* [T, 2] their softmax probabilities                */
+  int32_t* counts;     /* [E]    token slots per expert                     */
+  int32_t* offsets;    /* [E+1]  exclusive prefix of counts                 */
+  int32_t* perm_token; /* [2T]   token of each permuted row                 */
+  int32_t* perm_slot;  /* [2T]   slot (0/1) of each permuted row            */
+  void* h;             /* [2T, f] x-dtype: GELU(x.Wg)*(x.Wu) per permuted row;
+                          when set, the kernels write the intermediate here   */
+} moe_debug_t;
+
+/* Forward pass with a library-owned workspace: one cache per device, grown
+ * with cudaMalloc when a call needs more (never shrunk), guarded by a mutex.
+ * Calls on one device share that workspace, so calls that may overlap on the
+ * GPU (different streams) must use moe_forward_ex with their own workspaces.
+ * Returns MOE_OK or an error status (see the file header). */
+MOE_EXPORT moe_status_t moe_forward(const void* x, const float* w_router, const void* w_gate,
+                         const void* w_up, const void* w_down,
+                         const moe_scales_t* w_scales, void* out,
+                         int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
+                         moe_dtype_t dtype, moe_stream_t stream);
+
+/* Bytes of device workspace moe_forward_ex needs for these sizes (0 on bad
+ * arguments). `path` and `down_splits` as in moe_options_t (0 = auto). */
+MOE_EXPORT size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
+                          moe_dtype_t dtype, moe_path_t path, int32_t down_splits);
+
+/* Forward pass on a caller-provided device workspace of ws_bytes bytes
+ * (256-byte aligned, at least moe_workspace_size(...)); allocates nothing.
+ * `opts` and `dbg` may be NULL. Concurrent calls need distinct workspaces. */
+MOE_EXPORT moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options_t* opts,
+                            const moe_debug_t* dbg, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* Synchronises `stream` and reads the status word that the kernels of the last
+ * call on `workspace` recorded (NULL = the moe_forward cache of the current
+ * device). Returns MOE_OK, MOE_ERR_DEVICE_CHECK (and the raw code in *code if
+ * code != NULL) or MOE_ERR_CUDA. */
+MOE_EXPORT moe_status_t moe_device_status(const void* workspace, moe_stream_t stream, uint32_t* code);
+
+/* Static description of a status code (never NULL). */
+MOE_EXPORT const char* moe_status_string(moe_status_t status);
+
+/* Library ABI version, currently 1. */
+MOE_EXPORT int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

@@ -1,0 +1,133 @@
+"""B200 (sm_100a) Grok-1 MoE feed-forward sublayer: Python binding of the C ABI.
+
+Functions carry the C names (include/moe.h) and take torch CUDA tensors; they
+only marshal arguments into ``libmoe_b200.so``. Errors raise ``MoeError``.
+
+    import torch, mixture_experts_ffn_14_b200 as moe
+    out = torch.empty_like(x)
+    moe.moe_forward(x, w_router, w_gate, w_up, w_down, out)
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+from . import _native as N
+from ._native import (  # noqa: F401
+    MOE_BF16, MOE_BF16_INT8W, MOE_F32, MOE_GELU_ERF, MOE_GELU_TANH, MOE_PATH_AUTO,
+    MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM,
+)
+
+__all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_workspace_size", "moe_device_status",
+           "moe_status_string", "moe_abi_version", "dtype_code"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {moe_status_string(status)} (status {status})")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("moe: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("moe: tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def dtype_code(x, w_gate) -> int:
+    import torch
+
+    if w_gate.dtype == torch.int8:
+        return MOE_BF16_INT8W
+    if x.dtype == torch.float32:
+        return MOE_F32
+    return MOE_BF16
+
+
+def _scales(scales):
+    if scales is None:
+        return None
+    sg, su, sd = scales
+    return N.MoeScales(_ptr(sg), _ptr(su), _ptr(sd))
+
+
+def moe_status_string(status: int) -> str:
+    return N.lib().moe_status_string(status).decode()
+
+
+def moe_abi_version() -> int:
+    return N.lib().moe_abi_version()
+
+
+def moe_workspace_size(T, d, f, E=8, k=2, dtype=MOE_BF16, path=MOE_PATH_AUTO, down_splits=0) -> int:
+    return N.lib().moe_workspace_size(T, d, f, E, k, dtype, path, down_splits)
+
+
+def moe_forward(x, w_router, w_gate, w_up, w_down, out, scales=None, stream=None):
+    """out[T, d] = MoE FFN of x[T, d] (library-owned workspace)."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    sc = _scales(scales)
+    st = N.lib().moe_forward(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                             ctypes.byref(sc) if sc is not None else None, _ptr(out),
+                             T, d, f, E, 2, dtype_code(x, w_gate), _stream(stream))
+    if st != N.MOE_OK:
+        raise MoeError(st, "moe_forward")
+    return out
+
+
+def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=None, router_bias=None,
+                   gelu=MOE_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, debug=None, stream=None,
+                   stage_events=None, raise_on_error=True):
+    """Forward pass on a caller workspace (a uint8 CUDA tensor). ``debug`` is a
+    dict with any of idx, gates, counts, offsets, perm_token, perm_slot, h.
+    ``stage_events``: 6 torch.cuda.Event (already created, e.g. recorded once)
+    that the library records around its five stages."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    sc = _scales(scales)
+    args = N.MoeArgs(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                     ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
+                     dtype_code(x, w_gate))
+    ev = None
+    if stage_events is not None:
+        handles = [e.cuda_event for e in stage_events]
+        if len(handles) != 6 or not all(handles):
+            raise ValueError("moe: stage_events needs 6 created CUDA events")
+        ev = (ctypes.c_void_p * 6)(*handles)
+    opts = N.MoeOptions(gelu, _ptr(router_bias), path, down_splits,
+                        ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)) if ev is not None else None)
+    dbg = None
+    if debug:
+        dbg = N.MoeDebug(*[_ptr(debug.get(n)) for n in
+                           ("idx", "gates", "counts", "offsets", "perm_token", "perm_slot", "h")])
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = N.lib().moe_forward_ex(ctypes.byref(args), ctypes.byref(opts),
+                                ctypes.byref(dbg) if dbg is not None else None,
+                                _ptr(workspace), ws_bytes, _stream(stream))
+    if st != N.MOE_OK and raise_on_error:
+        raise MoeError(st, "moe_forward_ex")
+    return st
+
+
+def moe_device_status(workspace=None, stream=None):
+    """(status, code) recorded by the kernels of the last call on ``workspace``."""
+    code = ctypes.c_uint32(0)
+    st = N.lib().moe_device_status(_ptr(workspace), _stream(stream), ctypes.byref(code))
+    return st, code.value

@@ -1,0 +1,74 @@
+"""ctypes binding of ``libmoe_b200.so`` (the C ABI declared in include/moe.h).
+
+Argument marshalling only: every step of the forward pass runs in the
+library's CUDA kernels. There is no fallback: if the library is missing or a
+call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 3
+MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK = 4, 5, 6
+MOE_F32, MOE_BF16, MOE_BF16_INT8W = 0, 1, 2
+MOE_GELU_TANH, MOE_GELU_ERF = 0, 1
+MOE_PATH_AUTO, MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM = 0, 1, 2
+
+# Every function include/moe.h exports, with (restype, argtypes).
+EXPORTS = {}
+
+
+class MoeScales(ctypes.Structure):
+    _fields_ = [("s_gate", c_void_p), ("s_up", c_void_p), ("s_down", c_void_p)]
+
+
+class MoeArgs(ctypes.Structure):
+    _fields_ = [("x", c_void_p), ("w_router", c_void_p), ("w_gate", c_void_p), ("w_up", c_void_p),
+                ("w_down", c_void_p), ("w_scales", POINTER(MoeScales)), ("out", c_void_p),
+                ("T", c_int64), ("d", c_int64), ("f", c_int64), ("E", c_int32), ("k", c_int32),
+                ("dtype", c_int)]
+
+
+class MoeOptions(ctypes.Structure):
+    _fields_ = [("gelu", c_int), ("router_bias", c_void_p), ("path", c_int), ("down_splits", c_int32),
+                ("stage_events", POINTER(c_void_p))]
+
+
+class MoeDebug(ctypes.Structure):
+    _fields_ = [("idx", c_void_p), ("gates", c_void_p), ("counts", c_void_p), ("offsets", c_void_p),
+                ("perm_token", c_void_p), ("perm_slot", c_void_p), ("h", c_void_p)]
+
+
+EXPORTS.update({
+    "moe_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(MoeScales), c_void_p,
+                            c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_void_p]),
+    "moe_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_int, c_int32]),
+    "moe_forward_ex": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), POINTER(MoeDebug), c_void_p, c_size_t,
+                               c_void_p]),
+    "moe_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_uint32)]),
+    "moe_status_string": (c_char_p, [c_int]),
+    "moe_abi_version": (c_int32, []),
+})
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library once; raise if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m mixture_experts_ffn_14_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB

@@ -1,0 +1,571 @@
+// gemm_sm100.cu — grouped expert GEMMs on the 5th-generation tensor cores.
+//
+// Two kernels share one persistent, warp-specialised pipeline:
+//   GATEUP: H[r, n] = GELU(Xp[r,:] . Wg[e][:, n]) * (Xp[r,:] . Wu[e][:, n])     (bf16 out)
+//   DOWN:   Y[s, r, n] = gate[r] * (H[r, kslice_s] . Wd[e][kslice_s, n])         (fp32 out)
+// for every permuted row r of expert e (rows are expert-contiguous after the
+// dispatch stage). This is the GeGLU expert of the Grok-1 MoE sublayer (Grok-1
+// book ch. 10, section 10.4, "GeGLU vs SwiGLU" box: down(act(up_1 x) * up_2 x)).
+//
+// Roles per CTA (one CTA per SM, persistent over a static tile list):
+//   warp 0      TMA producer: activation tile + weight tile per 64-deep K stage
+//   warp 1      TMEM allocator and tcgen05.mma issuer (one thread)
+//   warps 4..7  epilogue: tcgen05.ld from TMEM, GELU / gate / scale, global stores
+//   warps 8..11 (int8 weights only) convert the int8 stage to bf16 in shared memory
+//
+// Shared memory per stage: X tile [128 rows x 64 K] bf16, K-major, 128-B swizzle
+// (16 KB) and W tile = four chunks [64 K x 64 N] bf16, N(MN)-major, 128-B swizzle
+// (32 KB); weights are used in the caller's [E, K, N] layout without a repack.
+//
+// Orientation:
+//   TOKEN_TILE    MMA M = 128 token rows (A = X, K-major), N = 256 weight columns
+//                 (B = W, MN-major); one MMA per 16-deep K step.
+//   WEIGHT_STREAM MMA M = 128 weight columns (A = W, MN-major), N = tokens of the
+//                 tile rounded up to 16 (B = X, K-major); two MMAs per K step.
+//                 Used when experts hold few tokens: every weight byte is read
+//                 once, the down projection is split along K for parallelism.
+// TMEM: 512 columns = two accumulator buffers of 256 columns, so the epilogue of
+// one tile overlaps the main loop of the next.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "moe_internal.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace tc {
+
+using namespace moe::sm100;
+
+constexpr int BM = 128;                 // tile rows (tokens)
+constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swizzle row
+constexpr int X_BYTES = BM * BK * 2;    // 16 KB
+constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16
+constexpr int W_BYTES = 4 * WCHUNK;     // 32 KB
+constexpr int W8_BYTES = BK * 256;      // 16 KB int8 staging: two [64 K x 128 N] boxes
+constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
+
+enum { GATEUP = 0, DOWN = 1 };
+
+template <bool W8>
+struct Cfg {
+  static constexpr int STAGES = W8 ? 3 : 4;
+  static constexpr int STAGE_BYTES = X_BYTES + W_BYTES + (W8 ? W8_BYTES : 0);
+  static constexpr int THREADS = W8 ? 384 : 256;
+  static constexpr int BAR_BYTES = 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+};
+
+struct Params {
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* gate_perm;
+  const __nv_bfloat16* s0;
+  const __nv_bfloat16* s1;
+  void* out;
+  int64_t rows;          // total permuted rows (2T)
+  int64_t split_stride;  // elements between split-K partial buffers (DOWN)
+  int32_t K, N;
+  int32_t splits;
+  int32_t kb_per_split;  // 64-deep K blocks per tile
+  int32_t ntile;         // output columns per tile (128 GATEUP, 256 DOWN)
+  int32_t gelu_mode;
+  uint32_t* status;
+};
+
+struct SharedSched {
+  int32_t cnt[kE];
+  int32_t off[kE];
+  int32_t mt[kE];
+  int32_t pre[kE + 1];
+};
+
+struct Tile {
+  int e, row0, rows, n0, kb0;
+};
+
+__device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& p, int tile, Tile& t) {
+  if (tile >= s.pre[kE]) return false;
+  int e = 0;
+  while (tile >= s.pre[e + 1]) ++e;
+  const int local = tile - s.pre[e];
+  const int nt_count = p.N / p.ntile;
+  const int mt = local % s.mt[e];
+  const int rest = local / s.mt[e];
+  const int nt = rest % nt_count;
+  const int ks = rest / nt_count;
+  t.e = e;
+  t.row0 = s.off[e] + mt * BM;
+  t.rows = min(BM, s.cnt[e] - mt * BM);
+  t.n0 = nt * p.ntile;
+  t.kb0 = ks * p.kb_per_split;
+  return true;
+}
+
+__device__ __forceinline__ float gelu_f32(float z, int mode) {
+  if (mode == MOE_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  const float u = 0.7978845608028654f * (z + 0.044715f * z * z * z);
+  return 0.5f * z * (1.0f + tanhf(u));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four int8 values (one 32-bit word) -> four bf16 (two 32-bit words), exact:
+// flip the sign bit to get q + 128 in [1, 255], place it in the low mantissa
+// bits of 2^23, subtract 2^23 + 128 in fp32, then pack to bf16 (|q| <= 127 is
+// exact in bf16).
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
+  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
+  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
+  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
+  lo = pack_bf16x2(f0, f1);
+  hi = pack_bf16x2(f2, f3);
+}
+
+template <int KIND, bool WS, bool W8>
+__global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
+    moe_expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
+                           const __grid_constant__ CUtensorMap tm_w1, const Params p) {
+  using C = Cfg<W8>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-B swizzle atoms.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* bar_area = smem + STAGES * C::STAGE_BYTES;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* conv_bar = empty_bar + STAGES;
+  uint64_t* tfull_bar = conv_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  SharedSched* sched = reinterpret_cast<SharedSched*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&conv_bar[s], 128);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 128);
+    }
+    *abort_flag = 0;
+    int acc = 0;
+    const int nt_count = p.N / p.ntile;
+    for (int e = 0; e < kE; ++e) {
+      const int c = p.counts[e];
+      sched->cnt[e] = c;
+      sched->off[e] = p.offsets[e];
+      sched->mt[e] = (c + BM - 1) / BM;
+      sched->pre[e] = acc;
+      acc += sched->mt[e] * nt_count * p.splits;
+    }
+    sched->pre[kE] = acc;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w0);
+    if (KIND == GATEUP) tma_prefetch_desc(&tm_w1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      // Weight-stream tiles read each weight byte once: mark it evict-first so
+      // it does not push the reused activations out of L2.
+      const uint64_t wpolicy = policy_evict_first();
+      auto load_w = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int n, int k, int e) {
+        if (WS) tma_load_3d_hint(dst, map, bar, n, k, e, wpolicy);
+        else tma_load_3d(dst, map, bar, n, k, e);
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      Tile t;
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+        const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
+        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
+        const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
+        for (int kb = 0; kb < p.kb_per_split; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) || *abort_flag) {
+            atomicOr(p.status, kStatusProducerTimeout);
+            *abort_flag = 1;
+            goto producer_done;
+          }
+          uint8_t* xs = smem + stage * C::STAGE_BYTES;
+          uint8_t* ws = xs + X_BYTES;
+          uint8_t* w8 = ws + W_BYTES;
+          const int k0 = (t.kb0 + kb) * BK;
+          mbar_arrive_expect_tx(&full_bar[stage], xbytes + wbytes);
+          if (WS) {
+            for (int b = 0; b < nbox_x; ++b)
+              tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
+          } else {
+            tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
+          }
+          if (W8) {
+            if (KIND == GATEUP) {
+              load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+              load_w(w8 + W8_BYTES / 2, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
+            } else {
+              load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+              load_w(w8 + W8_BYTES / 2, &tm_w0, &full_bar[stage], t.n0 + 128, k0, t.e);
+            }
+          } else {
+            if (KIND == GATEUP) {
+              // chunks 0,1: gate columns n0..n0+127; chunks 2,3: up columns n0..n0+127
+              load_w(ws + 0 * WCHUNK, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+              load_w(ws + 1 * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64, k0, t.e);
+              load_w(ws + 2 * WCHUNK, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
+              load_w(ws + 3 * WCHUNK, &tm_w1, &full_bar[stage], t.n0 + 64, k0, t.e);
+            } else {
+              for (int j = 0; j < 4; ++j)
+                load_w(ws + j * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64 * j, k0, t.e);
+            }
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      Tile t;
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
+          atomicOr(p.status, kStatusMmaTimeout);
+          *abort_flag = 1;
+          goto mma_done;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256;
+        const uint32_t ntok = WS ? ((t.rows + 15) / 16) * 16 : 0;
+        const uint32_t idesc = WS ? idesc_bf16_f32(128, ntok, 1, 0) : idesc_bf16_f32(128, 256, 0, 1);
+        for (int kb = 0; kb < p.kb_per_split; ++kb) {
+          uint64_t* ready = W8 ? &conv_bar[stage] : &full_bar[stage];
+          if (!mbar_wait(ready, phase, kWaitLimitNs) || *abort_flag) {
+            atomicOr(p.status, kStatusMmaTimeout);
+            *abort_flag = 1;
+            goto mma_done;
+          }
+          tc_fence_after();
+          const uint32_t xs = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t ws = xs + X_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < BK / 16; ++k16) {
+            const uint32_t accum = (kb | k16) != 0;
+            // X: K-major, 8-row groups 1024 B apart; a 16-deep K step is 32 B
+            // inside the swizzled 128-B row.
+            const uint64_t xdesc = smem_desc_sw128(xs + k16 * 32, 16, 1024);
+            if (WS) {
+              // W as A: MN-major, 64-column chunks 8 KB apart (LBO), 8-deep K
+              // groups 1024 B apart (SBO); a 16-deep K step is 2048 B.
+              const uint64_t a0 = smem_desc_sw128(ws + k16 * 2048, WCHUNK, 1024);
+              const uint64_t a1 = smem_desc_sw128(ws + 2 * WCHUNK + k16 * 2048, WCHUNK, 1024);
+              umma_bf16(d_tmem, a0, xdesc, idesc, accum);
+              umma_bf16(d_tmem + 128, a1, xdesc, idesc, accum);
+            } else {
+              const uint64_t wdesc = smem_desc_sw128(ws + k16 * 2048, WCHUNK, 1024);
+              umma_bf16(d_tmem, xdesc, wdesc, idesc, accum);
+            }
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        umma_commit(&tfull_bar[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    mma_done:;
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ epilogue --
+    const int q = warp - 4;  // TMEM lanes 32q .. 32q+31
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    Tile t;
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, kWaitLimitNs) || *abort_flag) {
+        atomicOr(p.status, kStatusEpilogueTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * 256;
+      if (!WS) {
+        const int r = 32 * q + lane;
+        const bool valid = r < t.rows;
+        const int64_t row = t.row0 + r;
+        if (KIND == GATEUP) {
+          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
+              float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
+              if (W8) {
+                const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c + j;
+                g0 *= __bfloat162float(p.s0[sc]);
+                g1 *= __bfloat162float(p.s0[sc + 1]);
+                u0 *= __bfloat162float(p.s1[sc]);
+                u1 *= __bfloat162float(p.s1[sc + 1]);
+              }
+              packed[j / 2] = pack_bf16x2(gelu_f32(g0, p.gelu_mode) * u0, gelu_f32(g1, p.gelu_mode) * u1);
+            }
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            }
+          }
+        } else {
+          float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
+          const float gate = valid ? p.gate_perm[row] : 0.0f;
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tbase + c, v);
+            if (valid) {
+              float o[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                float a = __uint_as_float(v[j]);
+                if (W8) a *= __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + t.n0 + c + j]);
+                o[j] = a * gate;
+              }
+              float4* dst = reinterpret_cast<float4*>(yout + row * p.N + t.n0 + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            }
+          }
+        }
+      } else {
+        // Weight-stream: TMEM lane = output column, TMEM column = token.
+        const int ntok = ((t.rows + 15) / 16) * 16;
+        if (KIND == GATEUP) {
+          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
+          const int n = t.n0 + 32 * q + lane;
+          float sg = 1.0f, su = 1.0f;
+          if (W8) {
+            sg = __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + n]);
+            su = __bfloat162float(p.s1[static_cast<int64_t>(t.e) * p.N + n]);
+          }
+#pragma unroll 1
+          for (int c = 0; c < ntok; c += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c + j < t.rows) {
+                const float h = gelu_f32(__uint_as_float(g[j]) * sg, p.gelu_mode) * (__uint_as_float(u[j]) * su);
+                hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] = __float2bfloat16_rn(h);
+              }
+            }
+          }
+        } else {
+          float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
+          const int n_a = t.n0 + 32 * q + lane;
+          const int n_b = n_a + 128;
+          float sa = 1.0f, sb = 1.0f;
+          if (W8) {
+            sa = __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + n_a]);
+            sb = __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + n_b]);
+          }
+#pragma unroll 1
+          for (int c = 0; c < ntok; c += 32) {
+            uint32_t a[32], b[32];
+            tmem_ld32x2(tbase + c, tbase + 128 + c, a, b);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c + j < t.rows) {
+                const int64_t row = t.row0 + c + j;
+                const float gate = p.gate_perm[row];
+                yout[row * p.N + n_a] = __uint_as_float(a[j]) * sa * gate;
+                yout[row * p.N + n_b] = __uint_as_float(b[j]) * sb * gate;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  } else if (W8 && warp >= 8) {
+    // ----------------------------------------------- int8 -> bf16 convert --
+    // Staging: two int8 boxes [64 K][128 N] (row = 128 B). Target: four bf16
+    // chunks [64 K][64 N] with the 128-B swizzle (16-B unit u of row k stored at
+    // unit u ^ (k % 8)).
+    const int ct = threadIdx.x - 256;  // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    Tile t;
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+      for (int kb = 0; kb < p.kb_per_split; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) || *abort_flag) {
+          atomicOr(p.status, kStatusConvertTimeout);
+          *abort_flag = 1;
+          goto convert_done;
+        }
+        {
+          uint8_t* xs = smem + stage * C::STAGE_BYTES;
+          uint8_t* ws = xs + X_BYTES;
+          const uint8_t* w8 = ws + W_BYTES;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int seg = ct + 128 * it;   // 0..1023: 16-byte int8 segments
+            const int box = seg >> 9;        // 512 segments per box
+            const int k = (seg >> 3) & 63;   // row
+            const int c16 = seg & 7;         // 16-column group in the 128-wide row
+            const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (W8_BYTES / 2) + k * 128 + c16 * 16);
+            const int col = c16 * 16;        // 0..112
+            const int chunk = box * 2 + (col >> 6);
+            const int u = (col & 63) >> 3;   // 16-B unit of the bf16 row (even)
+            uint32_t o[8];
+            i8x4_to_bf16x4(src.x, o[0], o[1]);
+            i8x4_to_bf16x4(src.y, o[2], o[3]);
+            i8x4_to_bf16x4(src.z, o[4], o[5]);
+            i8x4_to_bf16x4(src.w, o[6], o[7]);
+            uint8_t* rowp = ws + chunk * WCHUNK + k * 128;
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&conv_bar[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  convert_done:;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int KIND, bool WS, bool W8>
+cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
+  using C = Cfg<W8>;
+  auto kern = moe_expert_gemm_kernel<KIND, WS, W8>;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (configured_device != dev) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    configured_device = dev;
+  }
+
+  CUtensorMap tm_x, tm_w0, tm_w1;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.rows)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
+    const uint32_t box[2] = {BK, static_cast<uint32_t>(WS ? XBOX_ROWS_WS : BM)};
+    if (!encode_tensor_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), kE};
+    const uint64_t esz = W8 ? 1 : 2;
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.N) * esz, static_cast<uint64_t>(a.N) * a.K * esz};
+    const uint32_t box[3] = {static_cast<uint32_t>(W8 ? 128 : 64), BK, 1};
+    const CUtensorMapDataType dt = W8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle sw = W8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!encode_tensor_map(&tm_w0, dt, 3, a.w0, dims, strides, box, sw)) return cudaErrorInvalidValue;
+    if (!encode_tensor_map(&tm_w1, dt, 3, KIND == GATEUP ? a.w1 : a.w0, dims, strides, box, sw))
+      return cudaErrorInvalidValue;
+  }
+
+  Params p;
+  p.counts = a.counts;
+  p.offsets = a.offsets;
+  p.gate_perm = a.gate_perm;
+  p.s0 = a.s0;
+  p.s1 = a.s1;
+  p.out = a.out;
+  p.rows = a.rows;
+  p.split_stride = a.rows * static_cast<int64_t>(a.N);
+  p.K = a.K;
+  p.N = a.N;
+  p.splits = KIND == DOWN ? a.splits : 1;
+  p.kb_per_split = a.K / BK / p.splits;
+  p.ntile = KIND == GATEUP ? 128 : 256;
+  p.gelu_mode = a.gelu_mode;
+  p.status = a.status;
+
+  // Upper bound of the tile count (the exact count is only known on device).
+  const int64_t mtiles_max = a.rows / BM + kE;
+  const int64_t tiles_max = mtiles_max * (a.N / p.ntile) * p.splits;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles_max, device_sm_count()));
+  kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_x, tm_w0, tm_w1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s) {
+  if (a.weight_stream)
+    return a.int8_weights ? tc::launch_one<tc::GATEUP, true, true>(a, s) : tc::launch_one<tc::GATEUP, true, false>(a, s);
+  return a.int8_weights ? tc::launch_one<tc::GATEUP, false, true>(a, s) : tc::launch_one<tc::GATEUP, false, false>(a, s);
+}
+
+cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s) {
+  if (a.weight_stream)
+    return a.int8_weights ? tc::launch_one<tc::DOWN, true, true>(a, s) : tc::launch_one<tc::DOWN, true, false>(a, s);
+  return a.int8_weights ? tc::launch_one<tc::DOWN, false, true>(a, s) : tc::launch_one<tc::DOWN, false, false>(a, s);
+}
+
+}  // namespace moe

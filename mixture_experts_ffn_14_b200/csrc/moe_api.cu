@@ -1,0 +1,384 @@
+// moe_api.cu — the C ABI (include/moe.h): argument checks, workspace planning,
+// TMA descriptor encoding and the launch sequence
+//   router -> dispatch -> expert gate/up GEMM -> expert down GEMM -> combine
+// on the caller's stream, with no host synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t act_bytes(moe_dtype_t dt) { return dt == MOE_F32 ? 4 : 2; }
+
+// Sizes and dtype only (no pointers).
+moe_status_t check_sizes(const moe_args_t* a) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  if (a->T < 0 || a->d <= 0 || a->f <= 0) return MOE_ERR_INVALID_ARG;
+  if (a->dtype != MOE_F32 && a->dtype != MOE_BF16 && a->dtype != MOE_BF16_INT8W) return MOE_ERR_INVALID_ARG;
+  if (a->E != kE || a->k != kK) return MOE_ERR_UNSUPPORTED;
+  if (a->T > (int64_t(1) << 24) || a->d > (int64_t(1) << 20) || a->f > (int64_t(1) << 20))
+    return MOE_ERR_UNSUPPORTED;
+  if (a->dtype == MOE_F32) {
+    if (a->d % 64 != 0 || a->f % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (a->d % 256 != 0 || a->f % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  }
+  // Largest row offset used by the kernels must stay in 32-bit TMA coordinates
+  // and the per-expert weight slab in 64-bit addressing.
+  if (2 * a->T * std::max(a->d, a->f) > (int64_t(1) << 40)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_args(const moe_args_t* a) {
+  const moe_status_t st = check_sizes(a);
+  if (st != MOE_OK || a->T == 0) return st;
+  if (!a->x || !a->w_router || !a->w_gate || !a->w_up || !a->w_down || !a->out) return MOE_ERR_INVALID_ARG;
+  if (a->dtype == MOE_BF16_INT8W) {
+    if (!a->w_scales || !a->w_scales->s_gate || !a->w_scales->s_up || !a->w_scales->s_down)
+      return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a->w_scales->s_gate) || !aligned16(a->w_scales->s_up) || !aligned16(a->w_scales->s_down))
+      return MOE_ERR_MISALIGNED;
+  }
+  if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->w_gate) || !aligned16(a->w_up) ||
+      !aligned16(a->w_down) || !aligned16(a->out))
+    return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+// Signature of cuTensorMapEncodeTiled (driver API), fetched at run time through
+// the runtime's entry-point query so the library needs no link-time libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+std::mutex g_cache_mu;
+struct DeviceCache {
+  void* ws = nullptr;
+  size_t bytes = 0;
+};
+std::vector<DeviceCache> g_cache;
+
+std::vector<int> g_sm_count;
+std::mutex g_sm_mu;
+
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(g_sm_mu);
+  if (static_cast<int>(g_sm_count.size()) <= dev) g_sm_count.resize(dev + 1, 0);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return false;
+  cuuint64_t gdim[5];
+  cuuint64_t gstride[4];
+  cuuint32_t bdim[5];
+  cuuint32_t estride[5];
+  for (uint32_t i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+  }
+  for (uint32_t i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
+  const CUresult r = g_encode(map, dt, rank, const_cast<void*>(base), gdim, gstride, bdim, estride,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool use_weight_stream(int64_t T, moe_path_t path) {
+  if (path == MOE_PATH_WEIGHT_STREAM) return true;
+  if (path == MOE_PATH_TOKEN_TILE) return false;
+  // Average 2T/8 token slots per expert: at <= 64 (T <= 256) a 128-row token
+  // tile would be mostly padding, while weight-stream tiles take the tokens on
+  // the MMA N side and read each weight byte once.
+  return T <= 256;
+}
+
+int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested) {
+  const int64_t kblocks = f / 64;
+  auto valid = [&](int64_t s) { return s >= 1 && kblocks % s == 0; };
+  if (requested > 0) return valid(requested) ? requested : -1;
+  // Enough tiles for ~10 waves over the SMs; keep >= 8 K blocks per split.
+  const int64_t base_tiles = ((2 * T) / 128 + kE) * (d / 256);
+  int64_t best = 1;
+  for (int64_t s = 1; s <= 64; ++s) {
+    if (!valid(s) || kblocks / s < 8) continue;
+    best = s;
+    if (base_tiles * s >= 10 * 148) break;
+  }
+  return static_cast<int32_t>(best);
+}
+
+WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtype, moe_path_t path,
+                               int32_t down_splits, bool h_external) {
+  WorkspaceLayout L{};
+  const int64_t rows = 2 * T;
+  L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
+  L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path);
+  L.splits = L.weight_stream ? choose_down_splits(T, d, f, down_splits) : 1;
+  // A requested split factor must divide the K blocks whichever path runs.
+  if (down_splits > 0 && choose_down_splits(T, d, f, down_splits) < 1) L.splits = -1;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.idx = take(sizeof(int32_t) * rows);
+  L.gates = take(sizeof(float) * rows);
+  L.hist = take(sizeof(int32_t) * L.nblk * kE);
+  L.counts = take(sizeof(int32_t) * kE);
+  L.offsets = take(sizeof(int32_t) * (kE + 1));
+  L.perm_token = take(sizeof(int32_t) * rows);
+  L.perm_slot = take(sizeof(int32_t) * rows);
+  L.slot_pos = take(sizeof(int32_t) * rows);
+  L.gate_perm = take(sizeof(float) * rows);
+  L.xp = take(act_bytes(dtype) * rows * d);
+  L.h = h_external ? 0 : take(act_bytes(dtype) * rows * f);
+  L.y = take(sizeof(float) * static_cast<size_t>(std::max(L.splits, 1)) * rows * d);
+  L.total = o;
+  return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_debug_t* dbg, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream) {
+  const moe_options_t defaults{MOE_GELU_TANH, nullptr, MOE_PATH_AUTO, 0, nullptr};
+  if (!o) o = &defaults;
+  if (o->gelu != MOE_GELU_TANH && o->gelu != MOE_GELU_ERF) return MOE_ERR_INVALID_ARG;
+  if (o->path != MOE_PATH_AUTO && o->path != MOE_PATH_TOKEN_TILE && o->path != MOE_PATH_WEIGHT_STREAM)
+    return MOE_ERR_INVALID_ARG;
+  if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
+  if (o->router_bias && !aligned16(o->router_bias)) return MOE_ERR_MISALIGNED;
+  const bool h_ext = dbg && dbg->h;
+  if (h_ext && !aligned16(dbg->h)) return MOE_ERR_MISALIGNED;
+  const WorkspaceLayout L = plan_workspace(a->T, a->d, a->f, a->dtype, o->path, o->down_splits, h_ext);
+  if (L.splits < 1) return MOE_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < L.total)
+    return MOE_ERR_WORKSPACE;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* gates = reinterpret_cast<float*>(ws + L.gates);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_token = reinterpret_cast<int32_t*>(ws + L.perm_token);
+  int32_t* perm_slot = reinterpret_cast<int32_t*>(ws + L.perm_slot);
+  int32_t* slot_pos = reinterpret_cast<int32_t*>(ws + L.slot_pos);
+  float* gate_perm = reinterpret_cast<float*>(ws + L.gate_perm);
+  void* xp = ws + L.xp;
+  void* h = h_ext ? dbg->h : static_cast<void*>(ws + L.h);
+  float* y = reinterpret_cast<float*>(ws + L.y);
+  const int64_t T = a->T, d = a->d, f = a->f;
+
+#define MOE_TRY(call)                                  \
+  do {                                                 \
+    if ((call) != cudaSuccess) return MOE_ERR_CUDA;    \
+  } while (0)
+
+  auto mark = [&](int i) {
+    return o->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(o->stage_events[i]), stream) : cudaSuccess;
+  };
+  MOE_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  MOE_TRY(mark(0));
+  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, idx, gates, hist, stream));
+  MOE_TRY(mark(1));
+  MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
+                          slot_pos, gate_perm, xp, stream));
+  MOE_TRY(mark(2));
+  if (a->dtype == MOE_F32) {
+    MOE_TRY(launch_f32_gateup(static_cast<const float*>(xp), static_cast<const float*>(a->w_gate),
+                              static_cast<const float*>(a->w_up), counts, offsets, T, d, f, o->gelu,
+                              static_cast<float*>(h), stream));
+    MOE_TRY(mark(3));
+    MOE_TRY(launch_f32_down(static_cast<const float*>(h), static_cast<const float*>(a->w_down), counts, offsets,
+                            gate_perm, T, d, f, y, stream));
+  } else {
+    const bool w8 = a->dtype == MOE_BF16_INT8W;
+    TcGemmArgs g{};
+    g.x = xp;
+    g.w0 = a->w_gate;
+    g.w1 = a->w_up;
+    g.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_gate) : nullptr;
+    g.s1 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_up) : nullptr;
+    g.counts = counts;
+    g.offsets = offsets;
+    g.gate_perm = gate_perm;
+    g.out = h;
+    g.rows = 2 * T;
+    g.K = static_cast<int32_t>(d);
+    g.N = static_cast<int32_t>(f);
+    g.splits = 1;
+    g.gelu_mode = o->gelu;
+    g.int8_weights = w8;
+    g.weight_stream = L.weight_stream;
+    g.status = status;
+    MOE_TRY(launch_tc_gateup(g, stream));
+    MOE_TRY(mark(3));
+    TcGemmArgs g2 = g;
+    g2.x = h;
+    g2.w0 = a->w_down;
+    g2.w1 = nullptr;
+    g2.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_down) : nullptr;
+    g2.s1 = nullptr;
+    g2.out = y;
+    g2.K = static_cast<int32_t>(f);
+    g2.N = static_cast<int32_t>(d);
+    g2.splits = L.splits;
+    MOE_TRY(launch_tc_down(g2, stream));
+  }
+  MOE_TRY(mark(4));
+  MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, a->out, stream));
+  MOE_TRY(mark(5));
+
+  if (dbg) {
+    auto cp = [&](void* dst, const void* src, size_t bytes) {
+      return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, stream) : cudaSuccess;
+    };
+    MOE_TRY(cp(dbg->idx, idx, sizeof(int32_t) * 2 * T));
+    MOE_TRY(cp(dbg->gates, gates, sizeof(float) * 2 * T));
+    MOE_TRY(cp(dbg->counts, counts, sizeof(int32_t) * kE));
+    MOE_TRY(cp(dbg->offsets, offsets, sizeof(int32_t) * (kE + 1)));
+    MOE_TRY(cp(dbg->perm_token, perm_token, sizeof(int32_t) * 2 * T));
+    MOE_TRY(cp(dbg->perm_slot, perm_slot, sizeof(int32_t) * 2 * T));
+  }
+#undef MOE_TRY
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options_t* opts, const moe_debug_t* dbg,
+                            void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  const moe_status_t st = check_args(args);
+  if (st != MOE_OK || args->T == 0) return st;
+  return run_forward(args, opts, dbg, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k, moe_dtype_t dtype,
+                          moe_path_t path, int32_t down_splits) {
+  moe_args_t a{};
+  a.T = T;
+  a.d = d;
+  a.f = f;
+  a.E = E;
+  a.k = k;
+  a.dtype = dtype;
+  if (T <= 0 || check_sizes(&a) != MOE_OK) return 0;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_TOKEN_TILE && path != MOE_PATH_WEIGHT_STREAM) return 0;
+  if (down_splits < 0) return 0;
+  const WorkspaceLayout L = plan_workspace(T, d, f, dtype, path, down_splits, false);
+  if (L.splits < 1) return 0;
+  return L.total;
+}
+
+moe_status_t moe_forward(const void* x, const float* w_router, const void* w_gate, const void* w_up,
+                         const void* w_down, const moe_scales_t* w_scales, void* out, int64_t T, int64_t d,
+                         int64_t f, int32_t E, int32_t k, moe_dtype_t dtype, moe_stream_t stream) {
+  moe_args_t a{x, w_router, w_gate, w_up, w_down, w_scales, out, T, d, f, E, k, dtype};
+  const moe_status_t st = check_args(&a);
+  if (st != MOE_OK || T == 0) return st;
+  const size_t need = moe_workspace_size(T, d, f, E, k, dtype, MOE_PATH_AUTO, 0);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  if (static_cast<int>(g_cache.size()) <= dev) g_cache.resize(dev + 1);
+  DeviceCache& c = g_cache[dev];
+  if (c.bytes < need) {
+    // The previous buffer may still be in use by queued work on any stream.
+    if (c.ws) {
+      if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+      cudaFree(c.ws);
+      c.ws = nullptr;
+      c.bytes = 0;
+    }
+    if (cudaMalloc(&c.ws, need) != cudaSuccess) {
+      c.ws = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    c.bytes = need;
+  }
+  return run_forward(&a, nullptr, nullptr, c.ws, c.bytes, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_device_status(const void* workspace, moe_stream_t stream, uint32_t* code) {
+  const void* ws = workspace;
+  if (!ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    if (static_cast<int>(g_cache.size()) <= dev || !g_cache[dev].ws) {
+      if (code) *code = 0;
+      return MOE_OK;
+    }
+    ws = g_cache[dev].ws;
+  }
+  uint32_t v = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (code) *code = v;
+  return v == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported size or configuration";
+    case MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_DEVICE_CHECK: return "device-side check failed (see moe_device_status code)";
+  }
+  return "unknown status";
+}
+
+int32_t moe_abi_version(void) { return 1; }
+
+}  // extern "C"

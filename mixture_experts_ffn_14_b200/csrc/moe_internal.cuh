@@ -1,0 +1,94 @@
+// moe_internal.cuh — declarations shared by the library's translation units:
+// workspace layout, device status bits and kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kE = 8;              // experts (this version)
+constexpr int kK = 2;              // experts per token
+constexpr int kRouteTokens = 32;   // tokens per router / dispatch CTA
+
+// Device status word bits (set with atomicOr; 0 = no failure recorded).
+enum : uint32_t {
+  kStatusProducerTimeout = 1u << 0,
+  kStatusMmaTimeout = 1u << 1,
+  kStatusEpilogueTimeout = 1u << 2,
+  kStatusConvertTimeout = 1u << 3,
+};
+
+// Byte offsets of the regions of one call's workspace (each 256-aligned).
+struct WorkspaceLayout {
+  size_t status, idx, gates, hist, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm;
+  size_t xp, h, y, total;
+  int64_t nblk;      // router / dispatch CTAs
+  int32_t splits;    // split-K factor of the down projection
+  bool weight_stream;
+};
+
+// Host: workspace layout for a call (valid arguments assumed).
+WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtype, moe_path_t path,
+                               int32_t down_splits, bool h_external);
+
+// Host: which kernel family a call uses.
+bool use_weight_stream(int64_t T, moe_path_t path);
+int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested);
+
+// ---- launchers (return cudaSuccess or the launch error) --------------------
+
+cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
+                          int64_t d, int32_t* idx, float* gates, int32_t* hist, cudaStream_t s);
+
+cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
+                            const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
+                            int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
+                            float* gate_perm, void* xp, cudaStream_t s);
+
+cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
+                           const int32_t* slot_pos, int64_t T, int64_t d, void* out, cudaStream_t s);
+
+// fp32 (SIMT) grouped expert GEMMs.
+cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,
+                              const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t gelu_mode,
+                              float* h, cudaStream_t s);
+cudaError_t launch_f32_down(const float* h, const float* wd, const int32_t* counts, const int32_t* offsets,
+                            const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, cudaStream_t s);
+
+// tcgen05 grouped expert GEMMs (bf16 or int8 weights).
+struct TcGemmArgs {
+  const void* x;            // [rows, K] bf16 activations (Xp or H), rows = 2T
+  const void* w0;           // [E, K, N] gate (GATEUP) or down (DOWN) weights, bf16 or int8
+  const void* w1;           // [E, K, N] up weights (GATEUP) or nullptr
+  const __nv_bfloat16* s0;  // int8: [E, N] scales of w0, else nullptr
+  const __nv_bfloat16* s1;  // int8: [E, N] scales of w1, else nullptr
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* gate_perm;   // DOWN: gate of each permuted row
+  void* out;                // GATEUP: H bf16 [rows, N]; DOWN: Y fp32 [splits, rows, N]
+  int64_t rows;             // 2T
+  int32_t K, N;
+  int32_t splits;           // DOWN split-K factor (1 for GATEUP)
+  int32_t gelu_mode;
+  bool int8_weights;
+  bool weight_stream;
+  uint32_t* status;
+};
+cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
+
+// Host: encode a TMA descriptor (driver entry point fetched once).
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
+
+int device_sm_count();
+
+}  // namespace moe

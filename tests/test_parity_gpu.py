@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the oracle.
+
+Routing indices, counts, offsets and the dispatch permutation must match
+bit for bit (tokens within 1e-6 of a probability tie may take any ordering the
+oracle lists as valid); gates within 2e-6; outputs and the GeGLU intermediate
+within |gpu - ref| <= 1e-2 + 2e-2 |ref|."""
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_14_b200 as moe
+from mixture_experts_ffn_14_b200 import workloads as W
+
+from _harness import full_check, np64, run_gpu
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def small_bf16(T, d=512, f=384, seed=5, int8=False, skew=False):
+    w = W.Workload("small", T, d, f, dtype="bf16_int8w" if int8 else "bf16", seed=seed, skew=skew)
+    return W.make_torch(w, DEV)
+
+
+def tiny_f32(seed=0, T=64, d=128, f=256):
+    p = W.make_numpy(T, d, f, seed=seed)
+    return {k: torch.from_numpy(v).to(DEV) for k, v in p.items()}
+
+
+# ------------------------------------------------------------------ fp32 --
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_f32_full_parity(seed):
+    inp = tiny_f32(seed)
+    gpu = run_gpu(inp)
+    full_check(inp, gpu)
+
+
+@pytest.mark.parametrize("T", [1, 3, 33, 200])
+def test_f32_ragged_token_counts(T):
+    inp = tiny_f32(seed=T, T=T, d=128, f=192)
+    full_check(inp, run_gpu(inp))
+
+
+def test_f32_erf_gelu():
+    inp = tiny_f32(seed=9)
+    full_check(inp, run_gpu(inp, gelu=moe.MOE_GELU_ERF), gelu_mode="erf")
+
+
+# ------------------------------------------------------------------ bf16 --
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_WEIGHT_STREAM])
+@pytest.mark.parametrize("T", [1, 37, 300, 1000])
+def test_bf16_parity_both_paths(T, path):
+    inp = small_bf16(T)
+    full_check(inp, run_gpu(inp, path=path))
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3])
+def test_bf16_weight_stream_split_k(splits):
+    inp = small_bf16(90, d=256, f=384)
+    full_check(inp, run_gpu(inp, path=moe.MOE_PATH_WEIGHT_STREAM, down_splits=splits))
+
+
+def test_bf16_long_k_pipeline_wrap():
+    # K = 2048 (32 stages of 64) wraps the 4-deep ring many times; 3 n-tiles.
+    inp = small_bf16(260, d=2048, f=384, seed=11)
+    full_check(inp, run_gpu(inp, path=moe.MOE_PATH_TOKEN_TILE))
+
+
+def test_bf16_skewed_with_empty_experts():
+    inp = small_bf16(700, seed=12)
+    # Router bias that sends every token to experts 0 and 1: six experts empty,
+    # two experts with 700 rows each (6 m-tiles, ragged tail).
+    inp["router_bias"] = torch.tensor([40.0, 30.0, 0, 0, 0, 0, 0, 0], device=DEV)
+    gpu = run_gpu(inp, path=moe.MOE_PATH_TOKEN_TILE)
+    assert list(gpu["counts"]) == [700, 700, 0, 0, 0, 0, 0, 0]
+    full_check(inp, gpu)
+
+
+def test_bf16_skew_bias_workload_small():
+    inp = small_bf16(2048, d=256, f=256, seed=13, skew=True)
+    gpu = run_gpu(inp)
+    share = gpu["counts"] / gpu["counts"].sum()
+    assert share[0] > 0.45
+    full_check(inp, gpu, tokens=np.arange(0, 2048, 7))
+
+
+def test_bf16_erf_gelu():
+    inp = small_bf16(130, seed=14)
+    full_check(inp, run_gpu(inp, gelu=moe.MOE_GELU_ERF), gelu_mode="erf")
+
+
+# ------------------------------------------------------------------ int8 --
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_WEIGHT_STREAM])
+@pytest.mark.parametrize("T", [5, 300])
+def test_int8_parity_both_paths(T, path):
+    inp = small_bf16(T, seed=21, int8=True)
+    full_check(inp, run_gpu(inp, path=path))
+
+
+def test_int8_unit_scales_equal_bf16_path():
+    # |q| <= 127 is exact in bf16, so int8 weights with unit scales must give
+    # bitwise the bf16 result on the same values.
+    inp = small_bf16(150, seed=22, int8=True)
+    for s in ("s_gate", "s_up", "s_down"):
+        inp[s] = torch.ones_like(inp[s])
+    a = run_gpu(inp, path=moe.MOE_PATH_TOKEN_TILE, want_h=False)
+    b_inp = dict(inp)
+    for w in ("w_gate", "w_up", "w_down"):
+        b_inp[w] = inp[w].to(torch.bfloat16)
+    for s in ("s_gate", "s_up", "s_down"):
+        del b_inp[s]
+    b = run_gpu(b_inp, path=moe.MOE_PATH_TOKEN_TILE, want_h=False)
+    assert np.array_equal(a["out"], b["out"])
+
+
+# ------------------------------------------------------- determinism etc --
+
+def test_bitwise_determinism_and_streams():
+    inp = small_bf16(333, seed=31)
+    a = run_gpu(inp)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run_gpu(inp, stream=s)
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["perm_token"], b["perm_token"])
+
+
+def test_moe_forward_library_workspace_matches_ex():
+    inp = small_bf16(257, seed=32)
+    out = torch.empty_like(inp["x"])
+    moe.moe_forward(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
+    torch.cuda.synchronize()
+    ref = run_gpu(inp, want_h=False)
+    assert np.array_equal(np64(out), ref["out"])
+    assert moe.moe_device_status() == (0, 0)
+
+
+def test_zero_tokens_is_a_noop():
+    inp = small_bf16(4, seed=33)
+    x0 = inp["x"][:0]
+    out = torch.empty((0, inp["x"].shape[1]), dtype=torch.bfloat16, device=DEV)
+    moe.moe_forward(x0, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
