@@ -38,6 +38,7 @@ def parse():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode (T=64) side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--cpu-sample", type=int, default=64, help="tokens in the timed oracle sample")
     return ap.parse_args()
 
@@ -253,6 +254,31 @@ def main():
                 "down_gemm": {"achieved": round(down_tflops, 1), "frac": round(down_tflops / peak_t, 4)}}
 
     # ---- end-to-end through moe_forward with pinned host buffers -------------
+    e2e = run_e2e(a, moe, inp, out, flush, dist, dev, world, flops) if not a.no_e2e else None
+
+    # ---- decode side measurement: same weights, T = 64 ------------------------
+    decode = None
+    if not a.no_decode:
+        decode = run_decode(a, moe, W, wl, inp, dev, pk)
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------
+    cpu = None
+    if not a.no_cpu_baseline and world == 1 and rank == 0:
+        rng = np.random.default_rng(0)
+        sample = np.sort(rng.choice(T, size=min(a.cpu_sample, T), replace=False))
+        dt, _ = oracle_sample(inp, sample)
+        cpu = {"value": round(12 * d * f * len(sample) / dt / 1e12, 6), "unit": "TFLOP/s",
+               "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{len(sample)} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s"}
+    return finish(a, rank, world, dist, K, T, t_max, value, tok_s, stage_ms, roofline, e2e, decode, cpu, clk,
+                  wall, workload_name)
+
+
+def run_e2e(a, moe, inp, out, flush, dist, dev, world, flops):
+    import torch
+
+    T, d = inp["x"].shape
+    K = a.steps
     x_host = inp["x"].cpu().pin_memory()
     out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(inp["x"])
@@ -281,57 +307,55 @@ def main():
         tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
-    e2e = {"value": round(world * K * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-           "api": "moe_forward (library workspace), pinned host x -> device -> pinned host out"}
+    return {"value": round(world * K * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+            "api": "moe_forward (library workspace), pinned host x -> device -> pinned host out"}
 
-    # ---- decode side measurement: same weights, T = 64 ------------------------
-    decode = None
-    if not a.no_decode:
-        Td = W.WORKLOADS["decode"].T
-        xd = W.make_x(wl, dev, Td, seed_name="x_decode")
-        wsd = torch.empty(moe.moe_workspace_size(Td, d, f), dtype=torch.uint8, device=dev)
-        outd = torch.empty((Td, d), dtype=torch.bfloat16, device=dev)
-        cnt = torch.empty(8, dtype=torch.int32, device=dev)
-        evd = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-        for evs in evd:
-            for e in evs:
-                e.record()
 
-        def dstep(events=None, dbg=None):
-            moe.moe_forward_ex(xd, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], outd, wsd,
-                               stage_events=events, debug=dbg)
+def run_decode(a, moe, W, wl, inp, dev, pk):
+    import torch
 
-        for _ in range(a.warmup):
-            dstep(dbg={"counts": cnt})
-        torch.cuda.synchronize()
-        touched = int((cnt > 0).sum().item())
-        for i in range(K):
-            dstep(evd[i])
-        torch.cuda.synchronize()
-        d_ms = statistics.mean(ev[0].elapsed_time(ev[5]) for ev in evd)
-        d_gu = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in evd)
-        d_dn = statistics.mean(ev[3].elapsed_time(ev[4]) for ev in evd)
-        wbytes = touched * 3 * d * f * 2
-        decode = {"workload": f"grok1-decode T={Td} d={d} f={f} bf16 (same weights)",
-                  "ms_per_step": round(d_ms, 4), "experts_touched": touched,
-                  "hbm_gbs": round(wbytes / (d_ms / 1e3) / 1e9, 1),
-                  "frac": round(wbytes / (d_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
-                  "gate_up_gbs": round(touched * 2 * d * f * 2 / (d_gu / 1e3) / 1e9, 1),
-                  "down_gbs": round(touched * d * f * 2 / (d_dn / 1e3) / 1e9, 1),
-                  "peak_gbs": pk["hbm_gbs"], "bytes_per_step": wbytes}
+    K = a.steps
+    d, f = wl.d, wl.f
+    Td = W.WORKLOADS["decode"].T
+    xd = W.make_x(wl, dev, Td, seed_name="x_decode")
+    wsd = torch.empty(moe.moe_workspace_size(Td, d, f), dtype=torch.uint8, device=dev)
+    outd = torch.empty((Td, d), dtype=torch.bfloat16, device=dev)
+    cnt = torch.empty(8, dtype=torch.int32, device=dev)
+    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for evs in evd:
+        for e in evs:
+            e.record()
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------
-    cpu = None
-    if not a.no_cpu_baseline and world == 1 and rank == 0:
-        rng = np.random.default_rng(0)
-        sample = np.sort(rng.choice(T, size=min(a.cpu_sample, T), replace=False))
-        dt, _ = oracle_sample(inp, sample)
-        cpu = {"value": round(12 * d * f * len(sample) / dt / 1e12, 6), "unit": "TFLOP/s",
-               "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{len(sample)} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s"}
+    def dstep(events=None, dbg=None):
+        moe.moe_forward_ex(xd, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], outd, wsd,
+                           stage_events=events, debug=dbg)
 
+    for _ in range(a.warmup):
+        dstep(dbg={"counts": cnt})
+    torch.cuda.synchronize()
+    touched = int((cnt > 0).sum().item())
+    for i in range(K):
+        dstep(evd[i])
+    torch.cuda.synchronize()
+    d_ms = statistics.mean(ev[0].elapsed_time(ev[5]) for ev in evd)
+    d_gu = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in evd)
+    d_dn = statistics.mean(ev[3].elapsed_time(ev[4]) for ev in evd)
+    wbytes = touched * 3 * d * f * 2
+    return {"workload": f"grok1-decode T={Td} d={d} f={f} bf16 (same weights)",
+            "ms_per_step": round(d_ms, 4), "experts_touched": touched,
+            "hbm_gbs": round(wbytes / (d_ms / 1e3) / 1e9, 1),
+            "frac": round(wbytes / (d_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+            "gate_up_gbs": round(touched * 2 * d * f * 2 / (d_gu / 1e3) / 1e9, 1),
+            "down_gbs": round(touched * d * f * 2 / (d_dn / 1e3) / 1e9, 1),
+            "stage_ms": {"gate_up_gemm": round(d_gu, 4), "down_gemm": round(d_dn, 4)},
+            "peak_gbs": pk["hbm_gbs"], "bytes_per_step": wbytes}
+
+
+def finish(a, rank, world, dist, K, T, t_max, value, tok_s, stage_ms, roofline, e2e, decode, cpu, clk, wall,
+           workload_name):
     clocks = clk.summary()
+    d, f = 6144, 32768
     line = {
         "metric": "MoE-layer TFLOP/s, Grok-1 prefill (tokens/s and decode HBM GB/s alongside)",
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
@@ -344,11 +368,12 @@ def main():
         "tokens_per_s": round(tok_s, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,
-        "e2e": e2e,
         "gpu_launches": 5 * K,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
         "wall_s_timed_region": round(wall, 3),
     }
+    if e2e:
+        line["e2e"] = e2e
     if decode:
         line["decode"] = decode
     if cpu:
