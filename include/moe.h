@@ -148,6 +148,22 @@ MOE_EXPORT moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options
                             const moe_debug_t* dbg, void* workspace, size_t ws_bytes,
                             moe_stream_t stream);
 
+/* Forward pass that allocates nothing: its scratch is a fixed 32 MiB device
+ * array owned by the library (one per device that loads it, held until the
+ * process exits). For callers that must not call cudaMalloc at run time, such
+ * as a framework that reserves all device memory in its own pool at start-up,
+ * or a latency-critical loop where an allocation would stall the device. The
+ * pages have no counterpart: this is a deployment variant of moe_forward_ex.
+ * Same arguments and results as moe_forward_ex without workspace and debug
+ * outputs. With opts->down_splits == 0 the split-K factor is lowered until the
+ * scratch fits. Returns MOE_ERR_WORKSPACE when the problem needs more than the
+ * 32 MiB maximum (e.g. T = 64 at d = 6144, f = 32768 fits; T = 4096 does not).
+ * The first call on a device looks up the array's device address and should
+ * come before any stream capture. All calls on a device share the array:
+ * calls that may overlap on the GPU race and must be ordered by the caller. */
+MOE_EXPORT moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_options_t* opts,
+                                            moe_stream_t stream);
+
 /* Synchronises `stream` and reads the status word that the kernels of the last
  * call on `workspace` recorded (NULL = the moe_forward cache of the current
  * device). Returns MOE_OK, MOE_ERR_DEVICE_CHECK (and the raw code in *code if

@@ -18,8 +18,8 @@ from ._native import (  # noqa: F401
     MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM,
 )
 
-__all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_workspace_size", "moe_device_status",
-           "moe_status_string", "moe_abi_version", "dtype_code"]
+__all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_forward_noalloc", "moe_workspace_size",
+           "moe_device_status", "moe_status_string", "moe_abi_version", "dtype_code"]
 
 
 class MoeError(RuntimeError):
@@ -123,6 +123,28 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
                                 _ptr(workspace), ws_bytes, _stream(stream))
     if st != N.MOE_OK and raise_on_error:
         raise MoeError(st, "moe_forward_ex")
+    return st
+
+
+def moe_forward_noalloc(x, w_router, w_gate, w_up, w_down, out, scales=None, router_bias=None,
+                        gelu=MOE_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, stream=None,
+                        raise_on_error=True):
+    """Forward pass that allocates no device memory: the library runs it in a
+    fixed 32 MiB scratch array of its own, for callers that must not call
+    cudaMalloc while they run (e.g. a framework that owns all device memory in
+    a pre-reserved pool). Problems that need more scratch are rejected with
+    MOE_ERR_WORKSPACE. Calls on one device share the scratch, so calls that
+    may overlap on the GPU must be ordered by the caller."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    sc = _scales(scales)
+    args = N.MoeArgs(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                     ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
+                     dtype_code(x, w_gate))
+    opts = N.MoeOptions(gelu, _ptr(router_bias), path, down_splits, None)
+    st = N.lib().moe_forward_noalloc(ctypes.byref(args), ctypes.byref(opts), _stream(stream))
+    if st != N.MOE_OK and raise_on_error:
+        raise MoeError(st, "moe_forward_noalloc")
     return st
 
 

@@ -50,6 +50,7 @@ EXPORTS.update({
     "moe_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_int, c_int32]),
     "moe_forward_ex": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), POINTER(MoeDebug), c_void_p, c_size_t,
                                c_void_p]),
+    "moe_forward_noalloc": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), c_void_p]),
     "moe_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_uint32)]),
     "moe_status_string": (c_char_p, [c_int]),
     "moe_abi_version": (c_int32, []),

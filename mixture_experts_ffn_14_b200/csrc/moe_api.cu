@@ -382,3 +382,81 @@ const char* moe_status_string(moe_status_t s) {
 int32_t moe_abi_version(void) { return 1; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_forward_noalloc: the forward pass with its scratch in a fixed,
+// library-owned device array instead of memory the caller or the library
+// allocates at call time.
+//
+// Who needs it: code that must not call cudaMalloc while it runs, for example a
+// host framework that reserves all device memory in its own pool at start-up
+// (an allocation behind its back could fail late or break its accounting), or
+// a latency-critical loop where cudaMalloc / cudaFree would stall on a device
+// synchronisation. Such callers pass inputs and outputs only.
+//
+// The scratch is a static __device__ array of kNoAllocScratchBytes per device;
+// every GPU that loads this library holds it until the process exits. Host
+// code must not use the array's name as a device address (on the host it is
+// only a stand-in symbol), so the device address is fetched once per device
+// with cudaGetSymbolAddress while that device is current, on the first call
+// made on that device. That first call should therefore happen before any
+// stream capture. All calls on a device share the one array and leave their
+// contents in it: calls whose work may overlap on the GPU (different streams
+// without ordering) race on it. Each call clears the status word it uses; the
+// other scratch regions are fully written before they are read.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::vector<void*> g_noalloc_ptr;  // per device: device address of g_noalloc_scratch
+
+// Device address of the scratch array on the current device (set up once).
+cudaError_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (static_cast<int>(g_noalloc_ptr.size()) <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return err;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_options_t* opts,
+                                            moe_stream_t stream) {
+  const moe_status_t st = check_args(args);
+  if (st != MOE_OK || args->T == 0) return st;
+  moe_options_t o{MOE_GELU_TANH, nullptr, MOE_PATH_AUTO, 0, nullptr};
+  if (opts) o = *opts;
+  if (o.down_splits < 0) return MOE_ERR_INVALID_ARG;
+  WorkspaceLayout L = plan_workspace(args->T, args->d, args->f, args->dtype, o.path, o.down_splits, false);
+  if (L.splits < 1) return MOE_ERR_UNSUPPORTED;
+  if (L.total > kNoAllocScratchBytes && o.down_splits == 0 && L.splits > 1) {
+    // Automatic split-K: take the largest factor below the automatic one whose
+    // partial sums still fit the fixed scratch.
+    for (int32_t s = L.splits - 1; s >= 1; --s) {
+      const WorkspaceLayout C = plan_workspace(args->T, args->d, args->f, args->dtype, o.path, s, false);
+      if (C.splits == s && C.total <= kNoAllocScratchBytes) {
+        o.down_splits = s;
+        L = C;
+        break;
+      }
+    }
+  }
+  if (L.total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;  // problem too large for the fixed scratch
+  void* ws = nullptr;
+  if (noalloc_scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
+  return run_forward(args, &o, nullptr, ws, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
+}
