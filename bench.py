@@ -2,11 +2,13 @@
 """Benchmark of the Grok-1-shape MoE feed-forward sublayer on B200.
 
 One step = one forward of the whole sublayer (router, dispatch, gate/up GEMM,
-down GEMM, combine) over T = 4096 tokens, d = 6144, f = 32768, E = 8, top-2,
-bf16 activations and weights, fp32 router and accumulation. Inputs are seeded
-synthetic tensors already resident in HBM. Prints one JSON line.
+down GEMM, combine) over one batch, inputs already resident in HBM. The
+default workload is the Grok-1 prefill shape: T = 4096 tokens, d = 6144,
+f = 32768, E = 8, top-2, bf16 activations and weights, fp32 router and
+accumulation. Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                  [--workload prefill|decode|int8|skewed] [--T ..] [--d ..] [--f ..]
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica on its own GPU (the layer does not shard on this path): no data-path
@@ -17,6 +19,7 @@ ranks. `--impl reference` times the CPU oracle on the host cores instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -28,6 +31,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FLUSH_BYTES = 256 << 20           # > 126 MB L2
+METRIC = "MoE-layer TFLOP/s, Grok-1 prefill (tokens/s and decode HBM GB/s alongside)"
+STAGES = ["router", "dispatch", "gate_up_gemm", "down_gemm", "combine"]
 
 
 def parse():
@@ -36,6 +41,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", choices=["prefill", "decode", "int8", "skewed"], default="prefill")
+    ap.add_argument("--T", type=int, default=None, help="override the token count")
+    ap.add_argument("--d", type=int, default=None, help="override the hidden size")
+    ap.add_argument("--f", type=int, default=None, help="override the expert width")
+    ap.add_argument("--path", choices=["auto", "token_tile", "weight_stream", "token_tile_single"], default="auto",
+                    help="kernel family (default: the library's automatic choice)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode (T=64) side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
@@ -94,7 +105,7 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
+        sm, smax, power, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -103,6 +114,7 @@ class ClockSampler:
             try:
                 sm.append(float(parts[1]))
                 smax = float(parts[2])
+                power.append(float(parts[3]))
             except ValueError:
                 continue
             for n, v in zip(names, parts[5:9]):
@@ -111,29 +123,37 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
 # ------------------------------------------------------------ CPU oracle --
 
+def expert_getter(inp):
+    """One expert's matrices as float32 host arrays (exact for bf16; int8
+    weights dequantised by the oracle's own routine)."""
+    import oracle
+
+    def get(e):
+        if "s_gate" in inp:
+            return tuple(oracle.dequant_int8(inp[w][e].cpu().numpy(), inp[s][e].float().cpu().numpy())
+                         for w, s in (("w_gate", "s_gate"), ("w_up", "s_up"), ("w_down", "s_down")))
+        return tuple(inp[w][e].float().cpu().numpy() for w in ("w_gate", "w_up", "w_down"))
+    return get
+
+
 def oracle_sample(inp, tokens):
-    """Time the oracle (as it stands) on `tokens` of the workload; expert
-    matrices are copied from the device one expert at a time (float32, exact
-    for bf16) and the oracle converts them to float64 itself."""
+    """Time the oracle, as it stands, on `tokens` of the batch (routing of all
+    tokens included); the oracle converts each expert to float64 itself."""
     import numpy as np
 
     import oracle
 
     x = inp["x"].float().cpu().numpy()
     wr = inp["w_router"].float().cpu().numpy()
-
-    def get(e):
-        return tuple(inp[w][e].float().cpu().numpy() for w in ("w_gate", "w_up", "w_down"))
-
+    bias = inp["router_bias"].cpu().numpy() if "router_bias" in inp else None
     t0 = time.perf_counter()
-    res = oracle.forward_sparse(x, wr, get, tokens=np.asarray(tokens))
-    dt = time.perf_counter() - t0
-    return dt, res
+    oracle.forward_sparse(x, wr, expert_getter(inp), tokens=np.asarray(tokens), router_bias=bias)
+    return time.perf_counter() - t0
 
 
 def blas_threads():
@@ -149,6 +169,79 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
+# --------------------------------------------------------------- helpers --
+
+def workload(a):
+    from mixture_experts_ffn_14_b200 import workloads as W
+
+    wl = W.WORKLOADS[a.workload]
+    over = {k: getattr(a, k) for k in ("T", "d", "f") if getattr(a, k) is not None}
+    if over:
+        wl = dataclasses.replace(wl, **over)
+    dt = {"bf16": "bf16", "bf16_int8w": "int8 weights + bf16 scales, bf16 activations"}[wl.dtype]
+    name = f"grok1-{wl.name} T={wl.T} d={wl.d} f={wl.f} E={wl.E} k={wl.k} {dt}"
+    if wl.skew:
+        name += ", router bias -> ~50/15/15/4x5 % of slots"
+    return wl, name
+
+
+class Runner:
+    """One forward through the C ABI (moe_forward_ex on a preallocated workspace)."""
+
+    PATHS = {"auto": 0, "token_tile": 1, "weight_stream": 2, "token_tile_single": 3}
+
+    def __init__(self, moe, inp, T, d, f, dev, path="auto"):
+        import torch
+
+        self.moe, self.inp = moe, inp
+        self.path = self.PATHS[path]
+        dt = moe.dtype_code(inp["x"], inp["w_gate"])
+        self.ws = torch.empty(moe.moe_workspace_size(T, d, f, dtype=dt, path=self.path), dtype=torch.uint8,
+                              device=dev)
+        self.scales = (inp["s_gate"], inp["s_up"], inp["s_down"]) if "s_gate" in inp else None
+
+    def __call__(self, x, out, events=None, debug=None):
+        i = self.inp
+        self.moe.moe_forward_ex(x, i["w_router"], i["w_gate"], i["w_up"], i["w_down"], out, self.ws,
+                                scales=self.scales, router_bias=i.get("router_bias"), stage_events=events,
+                                debug=debug, path=self.path)
+
+
+def timed_steps(run, x, out, K, flush, clk=None):
+    """K steps, each bracketed by CUDA events (and the library's stage events),
+    with an L2 flush before each step outside its events."""
+    import torch
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for evs in stage_ev:          # materialise the event handles
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    for i in range(K):
+        if flush is not None:
+            flush.zero_()
+        starts[i].record()
+        run(x, out, stage_ev[i])
+        ends[i].record()
+    torch.cuda.synchronize()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    stage_ms = {n: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev)
+                for j, n in enumerate(STAGES)}
+    return step_ms, stage_ms
+
+
+def max_over_ranks(v, dist, dev):
+    if dist is None:
+        return v
+    import torch
+
+    t = torch.tensor([v], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- main --
 
 def main():
@@ -156,22 +249,18 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-
-    import numpy as np
-    import torch
-
-    from mixture_experts_ffn_14_b200 import workloads as W
-
-    wl = W.WORKLOADS["prefill"]
-    flops = wl.flops
-    workload_name = f"grok1-prefill T={wl.T} d={wl.d} f={wl.f} E={wl.E} k={wl.k} bf16"
+    wl, workload_name = workload(a)
 
     if a.impl == "reference":
         if rank != 0:
             return 0
         return run_reference(a, wl, workload_name, world)
 
+    import numpy as np
+    import torch
+
     import mixture_experts_ffn_14_b200 as moe
+    from mixture_experts_ffn_14_b200 import workloads as W
 
     dist = None
     if world > 1:
@@ -185,187 +274,69 @@ def main():
     torch.cuda.set_device(dev)
     pk = peaks()
 
-    inp = W.make_torch(wl, dev)
     T, d, f = wl.T, wl.d, wl.f
-    ws = torch.empty(moe.moe_workspace_size(T, d, f), dtype=torch.uint8, device=dev)
+    inp = W.make_torch(wl, dev)
+    run = Runner(moe, inp, T, d, f, dev, a.path)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def step(events=None):
-        moe.moe_forward_ex(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws,
-                           stage_events=events)
+    counts = torch.empty(8, dtype=torch.int32, device=dev)
 
     for _ in range(a.warmup):
         flush.zero_()
-        step()
+        run(inp["x"], out, debug={"counts": counts})
     torch.cuda.synchronize()
-    st, code = moe.moe_device_status(ws)
+    st, code = moe.moe_device_status(run.ws)
     if st != 0:
         raise SystemExit(f"device status {st} code {code:#x}")
-
+    touched = int((counts > 0).sum().item())
+    expert_counts = [int(v) for v in counts.cpu().tolist()]
     K = a.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    for evs in stage_ev:          # materialise the event handles
-        for e in evs:
-            e.record()
-    torch.cuda.synchronize()
 
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     with ClockSampler(dev) as clk:
-        for i in range(K):
-            flush.zero_()                       # L2 flush, outside the step's events
-            starts[i].record()
-            step(stage_ev[i])
-            ends[i].record()
-        torch.cuda.synchronize()
+        step_ms, stage_ms = timed_steps(run, inp["x"], out, K, flush)
     wall = time.perf_counter() - wall0
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks = clk.summary()
 
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    stage_names = ["router", "dispatch", "gate_up_gemm", "down_gemm", "combine"]
-    stage_ms = {n: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev)
-                for j, n in enumerate(stage_names)}
-    t_max = total_ms
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-
+    t_max = max_over_ranks(sum(step_ms), dist, dev)
+    flops = wl.flops
     value = world * K * flops / (t_max / 1e3) / 1e12
     tok_s = world * K * T / (t_max / 1e3)
+    wbytes = touched * 3 * d * f * (1 if wl.dtype == "bf16_int8w" else 2)
+    roofline = roofline_entry(wl, pk, stage_ms, touched, clocks)
 
-    # dominant kernel: the gate/up GEMM (2/3 of the FLOPs)
-    gu_flops = 8 * T * d * f
-    gu_tflops = gu_flops / (stage_ms["gate_up_gemm"] / 1e3) / 1e12
-    down_tflops = (4 * T * d * f) / (stage_ms["down_gemm"] / 1e3) / 1e12
-    peak_t = pk["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "kernel": "moe_expert_gemm_kernel<GATEUP> (gate+up GEMM, GELU*up epilogue)",
-                "achieved": round(gu_tflops, 1), "peak": peak_t, "unit": "TFLOP/s",
-                "frac": round(gu_tflops / peak_t, 4), "traffic": None,
-                "peak_source": f"{pk['source']} bf16 sustained",
-                "down_gemm": {"achieved": round(down_tflops, 1), "frac": round(down_tflops / peak_t, 4)}}
-
-    # ---- end-to-end through moe_forward with pinned host buffers -------------
-    e2e = run_e2e(a, moe, inp, out, flush, dist, dev, world, flops) if not a.no_e2e else None
-
-    # ---- decode side measurement: same weights, T = 64 ------------------------
+    e2e = None if a.no_e2e else run_e2e(a, moe, inp, run, out, flush, dist, dev, world, flops)
     decode = None
-    if not a.no_decode:
+    if not a.no_decode and wl.name == "prefill" and a.T is None:
         decode = run_decode(a, moe, W, wl, inp, dev, pk)
-
-    # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------------
     cpu = None
     if not a.no_cpu_baseline and world == 1 and rank == 0:
         rng = np.random.default_rng(0)
         sample = np.sort(rng.choice(T, size=min(a.cpu_sample, T), replace=False))
-        dt, _ = oracle_sample(inp, sample)
+        dt = oracle_sample(inp, sample)
         cpu = {"value": round(12 * d * f * len(sample) / dt / 1e12, 6), "unit": "TFLOP/s",
                "cores": blas_threads(), "kind": "oracle",
                "sample": f"{len(sample)} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s"}
-    return finish(a, rank, world, dist, K, T, t_max, value, tok_s, stage_ms, roofline, e2e, decode, cpu, clk,
-                  wall, workload_name)
 
-
-def run_e2e(a, moe, inp, out, flush, dist, dev, world, flops):
-    import torch
-
-    T, d = inp["x"].shape
-    K = a.steps
-    x_host = inp["x"].cpu().pin_memory()
-    out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
-    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.moe_forward(x_dev, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
-        out_host.copy_(out, non_blocking=True)
-
-    for _ in range(a.warmup):
-        flush.zero_()
-        e2e_step()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    for i in range(K):
-        flush.zero_()
-        e_s[i].record()
-        e2e_step()
-        e_e[i].record()
-    torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    return {"value": round(world * K * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-            "api": "moe_forward (library workspace), pinned host x -> device -> pinned host out"}
-
-
-def run_decode(a, moe, W, wl, inp, dev, pk):
-    import torch
-
-    K = a.steps
-    d, f = wl.d, wl.f
-    Td = W.WORKLOADS["decode"].T
-    xd = W.make_x(wl, dev, Td, seed_name="x_decode")
-    wsd = torch.empty(moe.moe_workspace_size(Td, d, f), dtype=torch.uint8, device=dev)
-    outd = torch.empty((Td, d), dtype=torch.bfloat16, device=dev)
-    cnt = torch.empty(8, dtype=torch.int32, device=dev)
-    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    for evs in evd:
-        for e in evs:
-            e.record()
-
-    def dstep(events=None, dbg=None):
-        moe.moe_forward_ex(xd, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], outd, wsd,
-                           stage_events=events, debug=dbg)
-
-    for _ in range(a.warmup):
-        dstep(dbg={"counts": cnt})
-    torch.cuda.synchronize()
-    touched = int((cnt > 0).sum().item())
-    for i in range(K):
-        dstep(evd[i])
-    torch.cuda.synchronize()
-    d_ms = statistics.mean(ev[0].elapsed_time(ev[5]) for ev in evd)
-    d_gu = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in evd)
-    d_dn = statistics.mean(ev[3].elapsed_time(ev[4]) for ev in evd)
-    wbytes = touched * 3 * d * f * 2
-    return {"workload": f"grok1-decode T={Td} d={d} f={f} bf16 (same weights)",
-            "ms_per_step": round(d_ms, 4), "experts_touched": touched,
-            "hbm_gbs": round(wbytes / (d_ms / 1e3) / 1e9, 1),
-            "frac": round(wbytes / (d_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
-            "gate_up_gbs": round(touched * 2 * d * f * 2 / (d_gu / 1e3) / 1e9, 1),
-            "down_gbs": round(touched * d * f * 2 / (d_dn / 1e3) / 1e9, 1),
-            "stage_ms": {"gate_up_gemm": round(d_gu, 4), "down_gemm": round(d_dn, 4)},
-            "peak_gbs": pk["hbm_gbs"], "bytes_per_step": wbytes}
-
-
-def finish(a, rank, world, dist, K, T, t_max, value, tok_s, stage_ms, roofline, e2e, decode, cpu, clk, wall,
-           workload_name):
-    clocks = clk.summary()
-    d, f = 6144, 32768
     line = {
-        "metric": "MoE-layer TFLOP/s, Grok-1 prefill (tokens/s and decode HBM GB/s alongside)",
-        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
-        "ms_per_step": round(t_max / K, 4), "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": a.warmup, "ms_per_step": round(t_max / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) activations, N(0, 1/sqrt(fan_in)) random-init weights",
         "config": {"workload": workload_name, "T": T, "d": d, "f": f, "E": 8, "k": 2,
-                   "l2": "flushed (256 MB write) between steps, outside the step events; weights 9.66 GB > L2",
+                   "l2": "flushed (256 MB write) between steps, outside the step events; "
+                         f"weights {wbytes / 1e9:.2f} GB > L2",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "tokens_per_s": round(tok_s, 1),
+        "expert_slots": expert_counts,
+        "path": a.path,
+        "hbm_gbs_weights": round(world * K * wbytes / (t_max / 1e3) / 1e9, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,
         "gpu_launches": 5 * K,
@@ -385,6 +356,102 @@ def finish(a, rank, world, dist, K, T, t_max, value, tok_s, stage_ms, roofline, 
     return 0
 
 
+def roofline_entry(wl, pk, stage_ms, touched, clocks):
+    """The gate/up GEMM is the dominant kernel (2/3 of the FLOPs; in the
+    weight-stream form 2/3 of the weight bytes)."""
+    T, d, f = wl.T, wl.d, wl.f
+    at_max = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                  and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"])
+    peak_t = pk["bf16_tflops"] if at_max else pk["bf16_tflops_sustained"]
+    src = f"{pk['source']} bf16 {'burst (clocks at max during the run)' if at_max else 'sustained'}"
+    gu_ms, dn_ms = stage_ms["gate_up_gemm"], stage_ms["down_gemm"]
+    esz = 1 if wl.dtype == "bf16_int8w" else 2
+    if T <= 256:   # weight-stream form: HBM bound
+        gu_bytes = touched * 2 * d * f * esz
+        gu = gu_bytes / (gu_ms / 1e3) / 1e9
+        dn = touched * d * f * esz / (dn_ms / 1e3) / 1e9
+        return {"bound": "hbm", "kernel": "moe_expert_gemm_kernel<GATEUP, WEIGHT_STREAM>",
+                "achieved": round(gu, 1), "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gu / pk["hbm_gbs"], 4),
+                "traffic": None, "peak_source": f"{pk['source']} HBM copy",
+                "algorithmic_per_launch": gu_bytes,
+                "down_gemm": {"achieved": round(dn, 1), "frac": round(dn / pk["hbm_gbs"], 4)}}
+    gu = 8 * T * d * f / (gu_ms / 1e3) / 1e12
+    dn = 4 * T * d * f / (dn_ms / 1e3) / 1e12
+    return {"bound": "tensor", "kernel": "moe_expert_gemm_kernel<GATEUP, TOKEN_TILE> (GELU*up epilogue)",
+            "achieved": round(gu, 1), "peak": peak_t, "unit": "TFLOP/s", "frac": round(gu / peak_t, 4),
+            "traffic": None, "peak_source": src, "algorithmic_per_launch": 8 * T * d * f,
+            "down_gemm": {"achieved": round(dn, 1), "frac": round(dn / peak_t, 4)}}
+
+
+def run_e2e(a, moe, inp, run, out, flush, dist, dev, world, flops):
+    """Same metric through the public API with the batch in pinned host memory:
+    every timed step copies x in and the result out."""
+    import torch
+
+    T, d = inp["x"].shape
+    K = a.steps
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    plain = "s_gate" not in inp and "router_bias" not in inp
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        if plain:
+            moe.moe_forward(x_dev, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
+        else:
+            run(x_dev, out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(a.warmup):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        e_s[i].record()
+        e2e_step()
+        e_e[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dist, dev)
+    return {"value": round(world * K * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+            "api": ("moe_forward (library workspace)" if plain else "moe_forward_ex")
+                   + ", pinned host x -> device -> pinned host out"}
+
+
+def run_decode(a, moe, W, wl, inp, dev, pk):
+    """Decode batch (T = 64) on the same weights: the weight-stream form."""
+    import torch
+
+    K = a.steps
+    d, f = wl.d, wl.f
+    Td = W.WORKLOADS["decode"].T
+    xd = W.make_x(wl, dev, Td, seed_name="x_decode")
+    run = Runner(moe, inp, Td, d, f, dev)
+    outd = torch.empty((Td, d), dtype=torch.bfloat16, device=dev)
+    cnt = torch.empty(8, dtype=torch.int32, device=dev)
+    for _ in range(a.warmup):
+        run(xd, outd, debug={"counts": cnt})
+    torch.cuda.synchronize()
+    touched = int((cnt > 0).sum().item())
+    step_ms, stage_ms = timed_steps(run, xd, outd, K, None)
+    d_ms = statistics.mean(step_ms)
+    wbytes = touched * 3 * d * f * 2
+    return {"workload": f"grok1-decode T={Td} d={d} f={f} bf16 (same weights)",
+            "ms_per_step": round(d_ms, 4), "experts_touched": touched,
+            "hbm_gbs": round(wbytes / (d_ms / 1e3) / 1e9, 1),
+            "frac": round(wbytes / (d_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+            "gate_up_gbs": round(touched * 2 * d * f * 2 / (stage_ms["gate_up_gemm"] / 1e3) / 1e9, 1),
+            "down_gbs": round(touched * d * f * 2 / (stage_ms["down_gemm"] / 1e3) / 1e9, 1),
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "peak_gbs": pk["hbm_gbs"], "bytes_per_step": wbytes}
+
+
 def run_reference(a, wl, workload_name, world):
     """The oracle on the host cores, same metric: each step is the oracle's
     forward for 8 tokens that all route to one expert pair (so a step converts
@@ -399,14 +466,13 @@ def run_reference(a, wl, workload_name, world):
     inp = W.make_torch(wl, dev)
     x = inp["x"].float().cpu().numpy()
     wr = inp["w_router"].float().cpu().numpy()
-    r = oracle.route(x, wr)
+    bias = inp["router_bias"].cpu().numpy() if "router_bias" in inp else None
+    r = oracle.route(x, wr, bias)
     pairs = {}
     for t, (e0, e1) in enumerate(r["idx"]):
         pairs.setdefault((min(e0, e1), max(e0, e1)), []).append(t)
-    groups = [v[:8] for _, v in sorted(pairs.items()) if len(v) >= 8]
-
-    def get(e):
-        return tuple(inp[w][e].float().cpu().numpy() for w in ("w_gate", "w_up", "w_down"))
+    groups = [v[:8] for _, v in sorted(pairs.items()) if len(v) >= 1]
+    get = expert_getter(inp)
 
     def one(i):
         toks = np.asarray(groups[i % len(groups)])
@@ -423,13 +489,14 @@ def run_reference(a, wl, workload_name, world):
         ntok += n
     v = 12 * wl.d * wl.f * ntok / total / 1e12
     line = {
-        "impl": "reference", "metric": "MoE-layer TFLOP/s, Grok-1 prefill (tokens/s and decode HBM GB/s alongside)",
+        "impl": "reference", "metric": METRIC,
         "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": round(total / a.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the b200 arm)",
         "config": {"workload": workload_name, "T": wl.T, "d": wl.d, "f": wl.f, "E": 8, "k": 2},
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": "per step 8 tokens routed to one expert pair (routing of all 4096 tokens done once)"},
+                         "sample": f"per step up to 8 tokens routed to one expert pair (routing of all {wl.T} "
+                                   "tokens done once)"},
         "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

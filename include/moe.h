@@ -75,8 +75,15 @@ typedef enum { MOE_GELU_TANH = 0, MOE_GELU_ERF = 1 } moe_gelu_t;
 
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
  * down projection) when the average tokens per expert is small, else
- * TOKEN_TILE (128-token tiles on the MMA M side). Both compute the same result. */
-typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_TOKEN_TILE = 1, MOE_PATH_WEIGHT_STREAM = 2 } moe_path_t;
+ * TOKEN_TILE (256-token tiles on the MMA M side of a CTA pair, cta_group::2).
+ * TOKEN_TILE_SINGLE runs 128-token tiles on single CTAs (kept for comparison).
+ * All compute the same result. */
+typedef enum {
+  MOE_PATH_AUTO = 0,
+  MOE_PATH_TOKEN_TILE = 1,
+  MOE_PATH_WEIGHT_STREAM = 2,
+  MOE_PATH_TOKEN_TILE_SINGLE = 3
+} moe_path_t;
 
 /* Per-output-channel scales of int8 weights (device pointers, bf16). */
 typedef struct {

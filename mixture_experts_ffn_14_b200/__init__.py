@@ -15,7 +15,7 @@ import ctypes
 from . import _native as N
 from ._native import (  # noqa: F401
     MOE_BF16, MOE_BF16_INT8W, MOE_F32, MOE_GELU_ERF, MOE_GELU_TANH, MOE_PATH_AUTO,
-    MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM,
+    MOE_PATH_TOKEN_TILE, MOE_PATH_TOKEN_TILE_SINGLE, MOE_PATH_WEIGHT_STREAM,
 )
 
 __all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_forward_noalloc", "moe_workspace_size",

@@ -17,7 +17,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK = 4, 5, 6
 MOE_F32, MOE_BF16, MOE_BF16_INT8W = 0, 1, 2
 MOE_GELU_TANH, MOE_GELU_ERF = 0, 1
-MOE_PATH_AUTO, MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM, MOE_PATH_TOKEN_TILE_SINGLE = 0, 1, 2, 3
 
 # Every function include/moe.h exports, with (restype, argtypes).
 EXPORTS = {}

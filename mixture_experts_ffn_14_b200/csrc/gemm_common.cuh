@@ -1,0 +1,240 @@
+// gemm_common.cuh — pieces shared by the single-CTA and the CTA-pair grouped
+// expert GEMM kernels: tile constants, parameters, the device-side tile
+// scheduler data, GELU, the exact int8 -> bf16 conversion and the token-tile
+// epilogue (GELU(gate) * up -> bf16 H, or gate * down -> fp32 Y).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "moe_internal.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace tc {
+
+using namespace moe::sm100;
+
+constexpr int BM = 128;                 // tile rows (tokens) per CTA
+constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swizzle row
+constexpr int X_BYTES = BM * BK * 2;    // 16 KB
+constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16, 128-B swizzle
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
+
+enum { GATEUP = 0, DOWN = 1 };
+
+struct Params {
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* gate_perm;
+  const __nv_bfloat16* s0;
+  const __nv_bfloat16* s1;
+  void* out;
+  int64_t rows;          // total permuted rows (2T)
+  int64_t split_stride;  // elements between split-K partial buffers (DOWN)
+  int32_t K, N;
+  int32_t splits;
+  int32_t kb_per_split;  // 64-deep K blocks per tile
+  int32_t ntile;         // output columns per tile (128 GATEUP, 256 DOWN)
+  int32_t gelu_mode;
+  int32_t select;        // kRunAlways, or run only if the pair / single form is preferred
+  int32_t sm_count;      // SMs of the device (same value for both token-tile kernels)
+  uint32_t* status;
+};
+
+enum { kRunAlways = 0, kRunIfPair = 1, kRunIfSingle = 2 };
+
+// Token tiles can run as 128-row tiles on single CTAs or as 256-row tiles on
+// CTA pairs. Which is faster depends on the per-expert counts (only known on
+// the device): pair tiles move a third less operand data per MMA but pad each
+// expert's row count up to a multiple of 256 instead of 128, and both forms
+// lose their last partial wave. Both kernels evaluate this on the same counts
+// and agree; the pair form is taken when its waves, discounted by 3 %, are fewer.
+__device__ __forceinline__ bool pair_preferred(const Params& p) {
+  int64_t single_tiles = 0, pair_tiles = 0;
+  for (int e = 0; e < kE; ++e) {
+    const int c = p.counts[e];
+    single_tiles += (c + 127) / 128;
+    pair_tiles += (c + 255) / 256;
+  }
+  const int64_t per = static_cast<int64_t>(p.N / p.ntile) * p.splits;
+  const int64_t sms = p.sm_count, pairs = p.sm_count / 2;
+  const int64_t w_single = (single_tiles * per + sms - 1) / sms;
+  const int64_t w_pair = (pair_tiles * per + pairs - 1) / pairs;
+  return w_pair * 100 < w_single * 103;
+}
+
+// True if this launch should do nothing (the other token-tile form runs).
+__device__ __forceinline__ bool skip_launch(const Params& p) {
+  if (p.select == kRunAlways) return false;
+  return pair_preferred(p) != (p.select == kRunIfPair);
+}
+
+struct SharedSched {
+  int32_t cnt[kE];
+  int32_t off[kE];
+  int32_t mt[kE];
+  int32_t pre[kE + 1];
+};
+
+struct Tile {
+  int e, row0, rows, n0, kb0;
+};
+
+// Row tiles of `tile_rows` per expert, column tiles of p.ntile, splits; row
+// tile fastest so that concurrently running CTAs share weight tiles in L2.
+__device__ __forceinline__ void build_sched(SharedSched& s, const Params& p, int tile_rows) {
+  int acc = 0;
+  const int nt_count = p.N / p.ntile;
+  for (int e = 0; e < kE; ++e) {
+    const int c = p.counts[e];
+    s.cnt[e] = c;
+    s.off[e] = p.offsets[e];
+    s.mt[e] = (c + tile_rows - 1) / tile_rows;
+    s.pre[e] = acc;
+    acc += s.mt[e] * nt_count * p.splits;
+  }
+  s.pre[kE] = acc;
+}
+
+__device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& p, int tile, int tile_rows,
+                                            Tile& t) {
+  if (tile >= s.pre[kE]) return false;
+  int e = 0;
+  while (tile >= s.pre[e + 1]) ++e;
+  const int local = tile - s.pre[e];
+  const int nt_count = p.N / p.ntile;
+  const int mt = local % s.mt[e];
+  const int rest = local / s.mt[e];
+  const int nt = rest % nt_count;
+  const int ks = rest / nt_count;
+  t.e = e;
+  t.row0 = s.off[e] + mt * tile_rows;
+  t.rows = min(tile_rows, s.cnt[e] - mt * tile_rows);
+  t.n0 = nt * p.ntile;
+  t.kb0 = ks * p.kb_per_split;
+  return true;
+}
+
+// Hardware tanh (PTX tanh.approx.f32, relative error ~2^-11): below the bf16
+// rounding that H receives right after, and a single instruction, which keeps
+// the epilogue from taking issue slots the int8 converters need.
+__device__ __forceinline__ float tanh_hw(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float gelu_f32(float z, int mode) {
+  if (mode == MOE_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  const float u = 0.7978845608028654f * (z + 0.044715f * z * z * z);
+  return 0.5f * z * (1.0f + tanh_hw(u));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four int8 values (one 32-bit word) -> four bf16 (two 32-bit words), exact:
+// flip the sign bit to get q + 128 in [1, 255], place it in the low mantissa
+// bits of 2^23, subtract 2^23 + 128 in fp32. An integer |q| <= 127 uses at most
+// the top 7 fraction bits of the fp32 result, so its low 16 bits are zero and
+// its high half is exactly the bf16 value: pack the high halves with a byte
+// permute (no rounding step needed).
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
+  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
+  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
+  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
+  lo = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
+  hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x7632);
+}
+
+// Convert 16-byte int8 segment `seg` of a staging area made of [64 K][128 N]
+// int8 boxes into the bf16 weight tile: box b covers bf16 chunks 2b and 2b+1,
+// each [64 K][64 N] with the 128-B swizzle (16-B unit u of row k is stored at
+// unit u ^ (k % 8)).
+__device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t* wtile, int seg) {
+  const int box = seg >> 9;        // 512 segments per box
+  const int k = (seg >> 3) & 63;   // row
+  const int c16 = seg & 7;         // 16-column group in the 128-wide row
+  const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (BK * 128) + k * 128 + c16 * 16);
+  const int col = c16 * 16;        // 0..112
+  const int chunk = box * 2 + (col >> 6);
+  const int u = (col & 63) >> 3;   // 16-B unit of the bf16 row (even)
+  uint32_t o[8];
+  i8x4_to_bf16x4(src.x, o[0], o[1]);
+  i8x4_to_bf16x4(src.y, o[2], o[3]);
+  i8x4_to_bf16x4(src.z, o[4], o[5]);
+  i8x4_to_bf16x4(src.w, o[6], o[7]);
+  uint8_t* rowp = wtile + chunk * WCHUNK + k * 128;
+  *reinterpret_cast<uint4*>(rowp + ((u ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Token-tile epilogue of one epilogue warp: TMEM lane = token row r (0..127 of
+// this CTA's rows starting at permuted row `row_base`), 256 accumulator
+// columns. GATEUP: columns 0..127 gate, 128..255 up -> bf16 H[row, n0 + c].
+// DOWN: 256 output columns -> fp32 Y[split, row, n0 + c] = acc * gate[row].
+template <int KIND, bool W8>
+__device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile& t, uint32_t tbase, int r,
+                                                    int64_t row_base, int nvalid) {
+  const bool valid = r < nvalid;
+  const int64_t row = row_base + r;
+  if (KIND == GATEUP) {
+    __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
+      uint32_t packed[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
+        float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
+        if (W8) {
+          const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c + j;
+          g0 *= __bfloat162float(p.s0[sc]);
+          g1 *= __bfloat162float(p.s0[sc + 1]);
+          u0 *= __bfloat162float(p.s1[sc]);
+          u1 *= __bfloat162float(p.s1[sc + 1]);
+        }
+        packed[j / 2] = pack_bf16x2(gelu_f32(g0, p.gelu_mode) * u0, gelu_f32(g1, p.gelu_mode) * u1);
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      }
+    }
+  } else {
+    float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
+    const float gate = valid ? p.gate_perm[row] : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+      uint32_t v[32];
+      tmem_ld32(tbase + c, v);
+      if (valid) {
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float a = __uint_as_float(v[j]);
+          if (W8) a *= __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + t.n0 + c + j]);
+          o[j] = a * gate;
+        }
+        float4* dst = reinterpret_cast<float4*>(yout + row * p.N + t.n0 + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      }
+    }
+  }
+}
+
+}  // namespace tc
+}  // namespace moe

@@ -11,7 +11,8 @@
 //   warp 0      TMA producer: activation tile + weight tile per 64-deep K stage
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one thread)
 //   warps 4..7  epilogue: tcgen05.ld from TMEM, GELU / gate / scale, global stores
-//   warps 8..11 (int8 weights only) convert the int8 stage to bf16 in shared memory
+//   warps 8..15 (int8 weights only) convert the int8 stage to bf16 in shared memory
+//               (two warps per SM sub-partition, so one hides the other's latency)
 //
 // Shared memory per stage: X tile [128 rows x 64 K] bf16, K-major, 128-B swizzle
 // (16 KB) and W tile = four chunks [64 K x 64 N] bf16, N(MN)-major, 128-B swizzle
@@ -33,104 +34,24 @@
 #include <algorithm>
 #include <cstdint>
 
-#include "moe_internal.cuh"
-#include "sm100.cuh"
+#include "gemm_common.cuh"
 
 namespace moe {
 namespace tc {
 
-using namespace moe::sm100;
-
-constexpr int BM = 128;                 // tile rows (tokens)
-constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swizzle row
-constexpr int X_BYTES = BM * BK * 2;    // 16 KB
-constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16
-constexpr int W_BYTES = 4 * WCHUNK;     // 32 KB
+constexpr int W_BYTES = 4 * WCHUNK;     // 32 KB: four [64 K x 64 N] chunks
 constexpr int W8_BYTES = BK * 256;      // 16 KB int8 staging: two [64 K x 128 N] boxes
 constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
-
-enum { GATEUP = 0, DOWN = 1 };
 
 template <bool W8>
 struct Cfg {
   static constexpr int STAGES = W8 ? 3 : 4;
   static constexpr int STAGE_BYTES = X_BYTES + W_BYTES + (W8 ? W8_BYTES : 0);
-  static constexpr int THREADS = W8 ? 384 : 256;
+  static constexpr int CONVERT_THREADS = 256;
+  static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : 256;
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
-
-struct Params {
-  const int32_t* counts;
-  const int32_t* offsets;
-  const float* gate_perm;
-  const __nv_bfloat16* s0;
-  const __nv_bfloat16* s1;
-  void* out;
-  int64_t rows;          // total permuted rows (2T)
-  int64_t split_stride;  // elements between split-K partial buffers (DOWN)
-  int32_t K, N;
-  int32_t splits;
-  int32_t kb_per_split;  // 64-deep K blocks per tile
-  int32_t ntile;         // output columns per tile (128 GATEUP, 256 DOWN)
-  int32_t gelu_mode;
-  uint32_t* status;
-};
-
-struct SharedSched {
-  int32_t cnt[kE];
-  int32_t off[kE];
-  int32_t mt[kE];
-  int32_t pre[kE + 1];
-};
-
-struct Tile {
-  int e, row0, rows, n0, kb0;
-};
-
-__device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& p, int tile, Tile& t) {
-  if (tile >= s.pre[kE]) return false;
-  int e = 0;
-  while (tile >= s.pre[e + 1]) ++e;
-  const int local = tile - s.pre[e];
-  const int nt_count = p.N / p.ntile;
-  const int mt = local % s.mt[e];
-  const int rest = local / s.mt[e];
-  const int nt = rest % nt_count;
-  const int ks = rest / nt_count;
-  t.e = e;
-  t.row0 = s.off[e] + mt * BM;
-  t.rows = min(BM, s.cnt[e] - mt * BM);
-  t.n0 = nt * p.ntile;
-  t.kb0 = ks * p.kb_per_split;
-  return true;
-}
-
-__device__ __forceinline__ float gelu_f32(float z, int mode) {
-  if (mode == MOE_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
-  const float u = 0.7978845608028654f * (z + 0.044715f * z * z * z);
-  return 0.5f * z * (1.0f + tanhf(u));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Four int8 values (one 32-bit word) -> four bf16 (two 32-bit words), exact:
-// flip the sign bit to get q + 128 in [1, 255], place it in the low mantissa
-// bits of 2^23, subtract 2^23 + 128 in fp32, then pack to bf16 (|q| <= 127 is
-// exact in bf16).
-__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t u = w ^ 0x80808080u;
-  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
-  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
-  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
-  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
-  lo = pack_bf16x2(f0, f1);
-  hi = pack_bf16x2(f2, f3);
-}
 
 template <int KIND, bool WS, bool W8>
 __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
@@ -151,6 +72,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   SharedSched* sched = reinterpret_cast<SharedSched*>(tmem_slot + 4);
 
+  if (skip_launch(p)) return;  // the other token-tile form takes this call
+
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -158,24 +81,14 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&conv_bar[s], 128);
+      mbar_init(&conv_bar[s], C::CONVERT_THREADS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 128);
     }
     *abort_flag = 0;
-    int acc = 0;
-    const int nt_count = p.N / p.ntile;
-    for (int e = 0; e < kE; ++e) {
-      const int c = p.counts[e];
-      sched->cnt[e] = c;
-      sched->off[e] = p.offsets[e];
-      sched->mt[e] = (c + BM - 1) / BM;
-      sched->pre[e] = acc;
-      acc += sched->mt[e] * nt_count * p.splits;
-    }
-    sched->pre[kE] = acc;
+    build_sched(*sched, p, BM);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -205,7 +118,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
         const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
         const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
         const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
@@ -262,7 +175,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusMmaTimeout);
           *abort_flag = 1;
@@ -320,7 +233,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
       if (!mbar_wait(&tfull_bar[acc], acc_phase, kWaitLimitNs) || *abort_flag) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
@@ -329,57 +242,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * 256;
       if (!WS) {
-        const int r = 32 * q + lane;
-        const bool valid = r < t.rows;
-        const int64_t row = t.row0 + r;
-        if (KIND == GATEUP) {
-          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
-            uint32_t g[32], u[32];
-            tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
-            uint32_t packed[16];
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
-              float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
-              if (W8) {
-                const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c + j;
-                g0 *= __bfloat162float(p.s0[sc]);
-                g1 *= __bfloat162float(p.s0[sc + 1]);
-                u0 *= __bfloat162float(p.s1[sc]);
-                u1 *= __bfloat162float(p.s1[sc + 1]);
-              }
-              packed[j / 2] = pack_bf16x2(gelu_f32(g0, p.gelu_mode) * u0, gelu_f32(g1, p.gelu_mode) * u1);
-            }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-            }
-          }
-        } else {
-          float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
-          const float gate = valid ? p.gate_perm[row] : 0.0f;
-#pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(tbase + c, v);
-            if (valid) {
-              float o[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                float a = __uint_as_float(v[j]);
-                if (W8) a *= __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + t.n0 + c + j]);
-                o[j] = a * gate;
-              }
-              float4* dst = reinterpret_cast<float4*>(yout + row * p.N + t.n0 + c);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-            }
-          }
-        }
+        epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, t.rows);
       } else {
         // Weight-stream: TMEM lane = output column, TMEM column = token.
         const int ntok = ((t.rows + 15) / 16) * 16;
@@ -440,11 +303,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     // Staging: two int8 boxes [64 K][128 N] (row = 128 B). Target: four bf16
     // chunks [64 K][64 N] with the 128-B swizzle (16-B unit u of row k stored at
     // unit u ^ (k % 8)).
-    const int ct = threadIdx.x - 256;  // 0..127
+    const int ct = threadIdx.x - 256;  // 0 .. CONVERT_THREADS-1
     int stage = 0;
     uint32_t phase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, t); tile += gridDim.x) {
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusConvertTimeout);
@@ -456,24 +319,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           uint8_t* ws = xs + X_BYTES;
           const uint8_t* w8 = ws + W_BYTES;
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int seg = ct + 128 * it;   // 0..1023: 16-byte int8 segments
-            const int box = seg >> 9;        // 512 segments per box
-            const int k = (seg >> 3) & 63;   // row
-            const int c16 = seg & 7;         // 16-column group in the 128-wide row
-            const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (W8_BYTES / 2) + k * 128 + c16 * 16);
-            const int col = c16 * 16;        // 0..112
-            const int chunk = box * 2 + (col >> 6);
-            const int u = (col & 63) >> 3;   // 16-B unit of the bf16 row (even)
-            uint32_t o[8];
-            i8x4_to_bf16x4(src.x, o[0], o[1]);
-            i8x4_to_bf16x4(src.y, o[2], o[3]);
-            i8x4_to_bf16x4(src.z, o[4], o[5]);
-            i8x4_to_bf16x4(src.w, o[6], o[7]);
-            uint8_t* rowp = ws + chunk * WCHUNK + k * 128;
-            *reinterpret_cast<uint4*>(rowp + ((u ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-          }
+          for (int it = 0; it < 1024 / C::CONVERT_THREADS; ++it)
+            convert_int8_segment(w8, ws, ct + C::CONVERT_THREADS * it);
         }
         fence_proxy_async_smem();
         mbar_arrive(&conv_bar[stage]);
@@ -544,6 +391,8 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.kb_per_split = a.K / BK / p.splits;
   p.ntile = KIND == GATEUP ? 128 : 256;
   p.gelu_mode = a.gelu_mode;
+  p.select = a.select;
+  p.sm_count = device_sm_count();
   p.status = a.status;
 
   // Upper bound of the tile count (the exact count is only known on device).

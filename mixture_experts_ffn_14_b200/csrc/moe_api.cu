@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -122,11 +123,44 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, 
 
 bool use_weight_stream(int64_t T, moe_path_t path) {
   if (path == MOE_PATH_WEIGHT_STREAM) return true;
-  if (path == MOE_PATH_TOKEN_TILE) return false;
+  if (path == MOE_PATH_TOKEN_TILE || path == MOE_PATH_TOKEN_TILE_SINGLE) return false;
   // Average 2T/8 token slots per expert: at <= 64 (T <= 256) a 128-row token
   // tile would be mostly padding, while weight-stream tiles take the tokens on
   // the MMA N side and read each weight byte once.
   return T <= 256;
+}
+
+// Split-K factor of the token-tile down projection. Its tiles are long (K = f)
+// and few (rows/128 x d/256), so the last partial wave can idle most SMs. For
+// balanced loads (each expert pads on average half a tile) estimate, per split
+// factor s, the time of the waves of whichever tile form the kernels will pick
+// (single-CTA 128-row tiles, or CTA-pair 256-row tiles at a 3 % discount), plus
+// 2.3 % of the unsplit work per extra split for the fp32 partial sums that are
+// written and read again (their bytes relative to the GEMM time at d, f).
+int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested, bool allow_single,
+                                      bool allow_pair) {
+  const int64_t kblocks = f / 64;
+  if (requested > 0) return kblocks % requested == 0 ? requested : -1;
+  auto valid = [&](int64_t s) { return s >= 1 && kblocks % s == 0 && kblocks / s >= 8; };
+  const double per_expert = static_cast<double>(2 * T) / kE;
+  const double nt = static_cast<double>(d / 256);
+  const double t1 = kE * (per_expert / 128.0 + 0.5) * nt;  // expected single-CTA tiles
+  const double t2 = kE * (per_expert / 256.0 + 0.5) * nt;  // expected pair tiles
+  const double sms = device_sm_count(), pairs = sms / 2;
+  int32_t best = 1;
+  double best_t = 1e30;
+  for (int64_t s = 1; s <= 8; ++s) {
+    if (!valid(s)) continue;
+    double t = 1e30;
+    if (allow_single) t = std::min(t, std::ceil(t1 * s / sms) / s);
+    if (allow_pair) t = std::min(t, std::ceil(t2 * s / pairs) / s / 1.03);
+    t += 0.023 * (s - 1) * (t1 / sms);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = static_cast<int32_t>(s);
+    }
+  }
+  return best;
 }
 
 int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested) {
@@ -150,7 +184,16 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   const int64_t rows = 2 * T;
   L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
   L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path);
-  L.splits = L.weight_stream ? choose_down_splits(T, d, f, down_splits) : 1;
+  if (dtype == MOE_F32) {
+    L.splits = 1;
+  } else if (L.weight_stream) {
+    L.splits = choose_down_splits(T, d, f, down_splits);
+  } else {
+    // Which token-tile forms may run (see the launch logic in run_forward).
+    const bool allow_pair = path == MOE_PATH_TOKEN_TILE || (path == MOE_PATH_AUTO && dtype != MOE_BF16_INT8W);
+    const bool allow_single = path != MOE_PATH_TOKEN_TILE;
+    L.splits = choose_token_tile_down_splits(T, d, f, down_splits, allow_single, allow_pair);
+  }
   // A requested split factor must divide the K blocks whichever path runs.
   if (down_splits > 0 && choose_down_splits(T, d, f, down_splits) < 1) L.splits = -1;
   size_t o = 0;
@@ -187,8 +230,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   const moe_options_t defaults{MOE_GELU_TANH, nullptr, MOE_PATH_AUTO, 0, nullptr};
   if (!o) o = &defaults;
   if (o->gelu != MOE_GELU_TANH && o->gelu != MOE_GELU_ERF) return MOE_ERR_INVALID_ARG;
-  if (o->path != MOE_PATH_AUTO && o->path != MOE_PATH_TOKEN_TILE && o->path != MOE_PATH_WEIGHT_STREAM)
-    return MOE_ERR_INVALID_ARG;
+  if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE) return MOE_ERR_INVALID_ARG;
   if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
   if (o->router_bias && !aligned16(o->router_bias)) return MOE_ERR_MISALIGNED;
   const bool h_ext = dbg && dbg->h;
@@ -256,7 +298,28 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.int8_weights = w8;
     g.weight_stream = L.weight_stream;
     g.status = status;
-    MOE_TRY(launch_tc_gateup(g, stream));
+    // Token tiles: with MOE_PATH_AUTO both forms are launched and the kernels
+    // pick one of them on the device from the expert counts (the other returns
+    // at once); TOKEN_TILE / TOKEN_TILE_SINGLE force one form.
+    // int8 weights always take single CTAs under AUTO: their pair form waits on
+    // both CTAs' converters every stage and measured slower.
+    const bool auto_tt = !L.weight_stream && o->path == MOE_PATH_AUTO && !w8;
+    const bool run_pair = !L.weight_stream && o->path != MOE_PATH_TOKEN_TILE_SINGLE &&
+                          !(w8 && o->path == MOE_PATH_AUTO);
+    const bool run_single = L.weight_stream || o->path != MOE_PATH_TOKEN_TILE;
+    auto launch_gemm = [&](TcGemmArgs args, bool down) -> cudaError_t {
+      if (run_pair) {
+        args.select = auto_tt ? 1 : 0;
+        const cudaError_t e = down ? launch_tc_down_pair(args, stream) : launch_tc_gateup_pair(args, stream);
+        if (e != cudaSuccess) return e;
+      }
+      if (run_single) {
+        args.select = auto_tt ? 2 : 0;
+        return down ? launch_tc_down(args, stream) : launch_tc_gateup(args, stream);
+      }
+      return cudaSuccess;
+    };
+    MOE_TRY(launch_gemm(g, false));
     MOE_TRY(mark(3));
     TcGemmArgs g2 = g;
     g2.x = h;
@@ -268,7 +331,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g2.K = static_cast<int32_t>(f);
     g2.N = static_cast<int32_t>(d);
     g2.splits = L.splits;
-    MOE_TRY(launch_tc_down(g2, stream));
+    MOE_TRY(launch_gemm(g2, true));
   }
   MOE_TRY(mark(4));
   MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, a->out, stream));
@@ -310,7 +373,7 @@ size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
   a.k = k;
   a.dtype = dtype;
   if (T <= 0 || check_sizes(&a) != MOE_OK) return 0;
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_TOKEN_TILE && path != MOE_PATH_WEIGHT_STREAM) return 0;
+  if (path < MOE_PATH_AUTO || path > MOE_PATH_TOKEN_TILE_SINGLE) return 0;
   if (down_splits < 0) return 0;
   const WorkspaceLayout L = plan_workspace(T, d, f, dtype, path, down_splits, false);
   if (L.splits < 1) return 0;

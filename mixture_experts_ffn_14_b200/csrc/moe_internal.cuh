@@ -79,10 +79,14 @@ struct TcGemmArgs {
   int32_t gelu_mode;
   bool int8_weights;
   bool weight_stream;
+  int32_t select;           // 0: always run; 1 / 2: run only if the pair / single token-tile form is preferred
   uint32_t* status;
 };
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
+// Token-tile form on CTA pairs (cta_group::2); `weight_stream` must be false.
+cudaError_t launch_tc_gateup_pair(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_tc_down_pair(const TcGemmArgs& a, cudaStream_t s);
 
 // Host: encode a TMA descriptor (driver entry point fetched once).
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const void* base,

@@ -50,9 +50,12 @@ def test_f32_erf_gelu():
 
 # ------------------------------------------------------------------ bf16 --
 
-@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_WEIGHT_STREAM])
+PATHS = [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE, moe.MOE_PATH_WEIGHT_STREAM]
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("T", [1, 37, 300, 1000])
-def test_bf16_parity_both_paths(T, path):
+def test_bf16_parity_all_paths(T, path):
     inp = small_bf16(T)
     full_check(inp, run_gpu(inp, path=path))
 
@@ -63,10 +66,31 @@ def test_bf16_weight_stream_split_k(splits):
     full_check(inp, run_gpu(inp, path=moe.MOE_PATH_WEIGHT_STREAM, down_splits=splits))
 
 
-def test_bf16_long_k_pipeline_wrap():
-    # K = 2048 (32 stages of 64) wraps the 4-deep ring many times; 3 n-tiles.
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE])
+@pytest.mark.parametrize("splits", [2, 3])
+def test_token_tile_split_k(path, splits):
+    for int8 in (False, True):
+        inp = small_bf16(400, d=512, f=384, seed=16, int8=int8)
+        full_check(inp, run_gpu(inp, path=path, down_splits=splits))
+
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE])
+def test_bf16_long_k_pipeline_wrap(path):
+    # K = 2048 (32 stages of 64) wraps the 4- and 6-deep rings many times; 3 n-tiles.
     inp = small_bf16(260, d=2048, f=384, seed=11)
-    full_check(inp, run_gpu(inp, path=moe.MOE_PATH_TOKEN_TILE))
+    full_check(inp, run_gpu(inp, path=path))
+
+
+@pytest.mark.parametrize("T", [1, 100, 129, 130, 255, 256, 257])
+def test_bf16_pair_tile_boundaries(T):
+    # Every token picks experts 0 and 1, so both hold T rows: the last 256-row
+    # pair tile leaves 0..128 valid rows to the second CTA of the pair.
+    inp = small_bf16(T, seed=15)
+    inp["router_bias"] = torch.tensor([40.0, 30.0, 0, 0, 0, 0, 0, 0], device=DEV)
+    for path in (moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE):
+        gpu = run_gpu(inp, path=path)
+        assert list(gpu["counts"][:2]) == [T, T]
+        full_check(inp, gpu)
 
 
 def test_bf16_skewed_with_empty_experts():
@@ -94,9 +118,9 @@ def test_bf16_erf_gelu():
 
 # ------------------------------------------------------------------ int8 --
 
-@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_WEIGHT_STREAM])
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("T", [5, 300])
-def test_int8_parity_both_paths(T, path):
+def test_int8_parity_all_paths(T, path):
     inp = small_bf16(T, seed=21, int8=True)
     full_check(inp, run_gpu(inp, path=path))
 
