@@ -8,6 +8,7 @@ fails loudly when the CUDA extension is missing instead of falling back.
 """
 
 from .moe_oracle import (  # noqa: F401
+    ACTIVATIONS,
     GELU_MODES,
     dequant_int8,
     dispatch,
@@ -18,7 +19,9 @@ from .moe_oracle import (  # noqa: F401
     gelu_erf,
     gelu_tanh,
     near_tie_mask,
+    post_norm_residual,
     route,
     route_alternatives,
+    silu,
     softmax_fp64,
 )

@@ -48,6 +48,14 @@ Readings where the pages are silent, ambiguous or disagree (each also in DESIGN.
       before the float32 rounding (used only to build the skewed-load workload).
   R7  int8 weights: W[e, i, j] = q[e, i, j] * s[e, j], one scale per output channel j
       ([ch1] INT8 box), dequantised here in float64.
+  R8  Mixtral-style routing ([ch10] §10.3.1 listing): the top-k probabilities divided
+      by their sum; this equals a softmax over the k selected logits, so the table's
+      "top-k -> softmax" and the listing's "softmax -> top-k -> renormalise" agree.
+      Its experts use SiLU (z * sigmoid(z)) on the gate branch ([ch10] §10.4 box).
+  R9  Sandwich post-norm ([ch10] §10.3.1: the post-RMSNorm compensates the gate sum
+      below 1; [blueprint] "MoE sublayer": the combined output is added back to the
+      trunk). The pages give no RMSNorm formula: the standard
+      w * y / sqrt(mean(y^2) + eps) over the hidden axis is used, eps a parameter.
 """
 
 from __future__ import annotations
@@ -57,7 +65,8 @@ from typing import Callable, Sequence
 
 import numpy as np
 
-GELU_MODES = ("tanh", "erf")
+ACTIVATIONS = ("tanh", "erf", "silu")
+GELU_MODES = ACTIVATIONS  # name kept for the GELU forms
 
 _SQRT_2_OVER_PI = math.sqrt(2.0 / math.pi)
 
@@ -80,12 +89,34 @@ def gelu_erf(z: np.ndarray) -> np.ndarray:
     return 0.5 * z * (1.0 + erf(z / math.sqrt(2.0)))
 
 
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU z * sigmoid(z), float64 (Mixtral experts, reading R8)."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
 def _gelu(z: np.ndarray, mode: str) -> np.ndarray:
     if mode == "tanh":
         return gelu_tanh(z)
     if mode == "erf":
         return gelu_erf(z)
-    raise ValueError(f"unknown gelu mode {mode!r}")
+    if mode == "silu":
+        return silu(z)
+    raise ValueError(f"unknown activation {mode!r}")
+
+
+def post_norm_residual(y, residual=None, weight=None, eps: float = 1e-5) -> np.ndarray:
+    """Sandwich post-norm and residual add of the sublayer output (reading R9):
+    out = residual + weight * y / sqrt(mean(y^2) + eps) over the last axis;
+    either part may be absent (weight None: no norm; residual None: no add)."""
+    y64 = np.asarray(y, dtype=np.float64)
+    out = y64
+    if weight is not None:
+        ms = np.mean(y64 * y64, axis=-1, keepdims=True)
+        out = np.asarray(weight, dtype=np.float64) * y64 / np.sqrt(ms + eps)
+    if residual is not None:
+        out = np.asarray(residual, dtype=np.float64) + out
+    return out
 
 
 def softmax_fp64(logits: np.ndarray) -> np.ndarray:
@@ -96,12 +127,13 @@ def softmax_fp64(logits: np.ndarray) -> np.ndarray:
     return e / np.sum(e, axis=-1, keepdims=True)
 
 
-def route(x, w_router, router_bias=None, k: int = 2) -> dict:
+def route(x, w_router, router_bias=None, k: int = 2, renormalize: bool = False) -> dict:
     """Router: logits = x . w_router (+ bias), rounded once to float32;
     probs = softmax(logits) in float64; top-k experts by descending logit
-    (ties -> lower index); gates = probs of the chosen experts, NOT renormalised.
+    (ties -> lower index); gates = probs of the chosen experts, NOT renormalised
+    (Grok-1), or divided by their sum with ``renormalize`` (Mixtral, reading R8).
 
-    [blueprint] "MoE sublayer"; [ch10] §10.3 table and §10.3.1; readings R3, R4, R6.
+    [blueprint] "MoE sublayer"; [ch10] §10.3 table and §10.3.1; readings R3, R4, R6, R8.
 
     x: [T, d]; w_router: [d, E]; router_bias: [E] or None.
     Returns dict with logits32 [T,E] float32, probs [T,E] float64,
@@ -119,6 +151,8 @@ def route(x, w_router, router_bias=None, k: int = 2) -> dict:
     order = np.argsort(-logits32, axis=1, kind="stable")
     idx = order[:, :k].astype(np.int32)
     gates = np.take_along_axis(probs, idx.astype(np.int64), axis=1)
+    if renormalize:  # Mixtral-style (reading R8)
+        gates = gates / np.sum(gates, axis=1, keepdims=True)
     return {"logits32": logits32, "probs": probs, "idx": idx, "gates": gates}
 
 
@@ -240,6 +274,7 @@ def forward_sparse(
     tokens: Sequence[int] | None = None,
     routing: dict | None = None,
     return_h: bool = False,
+    renormalize: bool = False,
 ) -> dict:
     """Sparse evaluation, expert by expert: out[t] = sum_s g_s * FFN_{e_s}(x[t]).
 
@@ -255,7 +290,7 @@ def forward_sparse(
     x = np.asarray(x)
     T = x.shape[0]
     if routing is None:
-        routing = route(x, w_router, router_bias, k)
+        routing = route(x, w_router, router_bias, k, renormalize)
     idx, gates = routing["idx"], routing["gates"]
     tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     get = _expert_getter(experts)
@@ -289,14 +324,14 @@ def forward_sparse(
 
 def forward_dense_bruteforce(
     x, w_router, experts, *, E: int = 8, k: int = 2, router_bias=None,
-    gelu_mode: str = "tanh",
+    gelu_mode: str = "tanh", renormalize: bool = False,
 ) -> np.ndarray:
     """Dense brute force, the way the published code does it ([ch11] §11.3.1
     item 3): evaluate all E experts on every token, then keep the top-k with a
     gate-weighted one-hot mask and sum over experts. float64."""
     x = np.asarray(x)
     T = x.shape[0]
-    routing = route(x, w_router, router_bias, k)
+    routing = route(x, w_router, router_bias, k, renormalize)
     mask = np.zeros((T, E), dtype=np.float64)
     for t in range(T):
         for s in range(k):

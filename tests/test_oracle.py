@@ -355,3 +355,56 @@ def test_bf16_rounding_helper():
     v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 3.14159], dtype=np.float32)
     ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float32).numpy()
     assert (workloads.round_bf16_np(v) == ref).all()
+
+
+# ------------------------------------------- next rows: Mixtral, post-norm --
+
+def test_renormalized_routing_closed_form_and_softmax_of_selected_logits():
+    g = _load("routing_closed_form.json")["renormalized_case"]
+    x = np.zeros((1, 8))
+    x[0, 0] = 1.0
+    wr = np.zeros((8, 8))
+    wr[0, :] = np.log(np.arange(1, 9, dtype=np.float64))
+    r = oracle.route(x, wr, renormalize=True)
+    assert list(r["idx"][0]) == g["idx"]
+    np.testing.assert_allclose(r["gates"][0], np.array(g["gates_num"]) / g["gates_den"], rtol=1e-6)
+    rng = np.random.default_rng(21)
+    xs = rng.standard_normal((100, 16))
+    wrs = rng.standard_normal((16, 8)) / 4
+    rr = oracle.route(xs, wrs, renormalize=True)
+    base = oracle.route(xs, wrs)
+    assert (rr["idx"] == base["idx"]).all()
+    sel = np.take_along_axis(rr["logits32"].astype(np.float64), rr["idx"].astype(np.int64), axis=1)
+    np.testing.assert_allclose(rr["gates"], scipy.special.softmax(sel, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(rr["gates"].sum(1), 1.0, rtol=1e-14)
+
+
+def test_silu_matches_library_and_mixtral_expert():
+    z = np.linspace(-30, 30, 3001)
+    ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
+    np.testing.assert_allclose(oracle.silu(z), ref, rtol=1e-13, atol=1e-15)
+    x, wr, wg, wu, wd = _rand_problem(T=6, d=16, f=24)
+    y, _ = oracle.expert_ffn(x, wg[1], wu[1], wd[1], "silu")
+    xt = torch.from_numpy(x)
+    lib = ((torch.nn.functional.silu(xt @ torch.from_numpy(wg[1])) * (xt @ torch.from_numpy(wu[1])))
+           @ torch.from_numpy(wd[1])).numpy()
+    np.testing.assert_allclose(y, lib, rtol=1e-12, atol=1e-14)
+    dense = oracle.forward_dense_bruteforce(x, wr, (wg, wu, wd), gelu_mode="silu", renormalize=True)
+    sparse = oracle.forward_sparse(x, wr, (wg, wu, wd), gelu_mode="silu", renormalize=True)["out"]
+    np.testing.assert_allclose(sparse, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_post_norm_matches_library_rms_norm():
+    rng = np.random.default_rng(22)
+    y = rng.standard_normal((7, 64)) * 0.3
+    w = rng.uniform(0.5, 1.5, 64)
+    res = rng.standard_normal((7, 64))
+    for eps in (1e-5, 1e-2):
+        lib = torch.nn.functional.rms_norm(torch.from_numpy(y), (64,), torch.from_numpy(w), eps=eps).numpy()
+        np.testing.assert_allclose(oracle.post_norm_residual(y, None, w, eps), lib, rtol=1e-12)
+        np.testing.assert_allclose(oracle.post_norm_residual(y, res, w, eps), res + lib, rtol=1e-12)
+    np.testing.assert_allclose(oracle.post_norm_residual(y, res), res + y, rtol=1e-15)
+    # A constant row c normalises to w * sign(c) / sqrt(1 + eps / c^2).
+    c = np.full((1, 64), -0.5)
+    out = oracle.post_norm_residual(c, None, w, 1e-5)
+    np.testing.assert_allclose(out[0], -w / np.sqrt(1 + 1e-5 / 0.25), rtol=1e-14)
