@@ -356,6 +356,29 @@ def main():
     return 0
 
 
+def recorded_traffic(wl):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu record,
+    or None when the workload differs or the GEMM sources changed since."""
+    import hashlib
+    import re
+
+    path = os.path.join(ROOT, "profiles", "gemm_traffic_prefill_T4096.md")
+    if not os.path.exists(path) or (wl.name, wl.T, wl.d, wl.f) != ("prefill", 4096, 6144, 32768):
+        return None
+    m = re.search(r"```json\n(.*?)\n```", open(path).read(), re.S)
+    if not m:
+        return None
+    rec = json.loads(m.group(1))
+    h = hashlib.sha256()
+    for src in rec["gemm_sources"]:
+        with open(os.path.join(ROOT, src), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["gemm_source_sha256"]:
+        return None
+    k = rec["kernels"]["gate_up"]
+    return k["dram_read_bytes"] + k["dram_write_bytes"]
+
+
 def roofline_entry(wl, pk, stage_ms, touched, clocks):
     """The gate/up GEMM is the dominant kernel (2/3 of the FLOPs; in the
     weight-stream form 2/3 of the weight bytes)."""
@@ -377,9 +400,11 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks):
                 "down_gemm": {"achieved": round(dn, 1), "frac": round(dn / pk["hbm_gbs"], 4)}}
     gu = 8 * T * d * f / (gu_ms / 1e3) / 1e12
     dn = 4 * T * d * f / (dn_ms / 1e3) / 1e12
-    return {"bound": "tensor", "kernel": "moe_expert_gemm_kernel<GATEUP, TOKEN_TILE> (GELU*up epilogue)",
+    return {"bound": "tensor",
+            "kernel": "gate/up expert GEMM, token tiles (single-CTA or CTA-pair form, chosen on the device)",
             "achieved": round(gu, 1), "peak": peak_t, "unit": "TFLOP/s", "frac": round(gu / peak_t, 4),
-            "traffic": None, "peak_source": src, "algorithmic_per_launch": 8 * T * d * f,
+            "traffic": recorded_traffic(wl), "peak_source": src, "algorithmic_per_launch": 8 * T * d * f,
+            "algorithmic_bytes_per_launch": wl.E * 2 * d * f * 2 + 2 * T * d * 2 + 2 * T * f * 2,
             "down_gemm": {"achieved": round(dn, 1), "frac": round(dn / peak_t, 4)}}
 
 

@@ -10,9 +10,15 @@
  *              lower expert index; gates g0 = p[e0], g1 = p[e1], NOT renormalised
  *     y_s    = ( GELU(x[t] . w_gate[e_s]) * (x[t] . w_up[e_s]) ) . w_down[e_s]
  *     out[t] = g0 * y_0 + g1 * y_1
- *   GELU is the tanh approximation unless MOE_GELU_ERF is asked for. Every
+ *   GELU is the tanh approximation unless MOE_ACT_GELU_ERF is asked for. Every
  *   routed (token, expert) pair is computed: no capacity limit, no token drop
  *   (Grok-1 book ch. 10, section 10.3.2, capacity-factor box).
+ * Options (moe_options_t) add the variants the same pages compare against:
+ *   renormalize = 1: gates divided by g0 + g1 (Mixtral, ch. 10 section 10.3.1);
+ *   MOE_ACT_SILU: SiLU instead of GELU on the gate branch (SwiGLU, section 10.4);
+ *   post_norm_weight / residual: out[t] = residual[t] + w * y / sqrt(mean(y^2) + eps)
+ *   with y the gate-weighted sum above, the sublayer's post-RMSNorm and residual
+ *   add (sandwich norm, section 10.3.1; the blueprint's "added back to the trunk").
  *
  * Pointers. Every array argument is a DEVICE pointer on the device that owns
  * `stream`; the caller owns all of them; the library never frees or retains
@@ -71,7 +77,12 @@ typedef enum {
   MOE_BF16_INT8W = 2   /* bf16 activations, int8 weights + bf16 channel scales */
 } moe_dtype_t;
 
-typedef enum { MOE_GELU_TANH = 0, MOE_GELU_ERF = 1 } moe_gelu_t;
+/* Activation on the gate branch of every expert. */
+typedef enum {
+  MOE_ACT_GELU_TANH = 0,  /* GELU, tanh approximation (default, Grok-1) */
+  MOE_ACT_GELU_ERF = 1,   /* GELU, z * Phi(z)                           */
+  MOE_ACT_SILU = 2        /* SiLU, z * sigmoid(z) (Mixtral)             */
+} moe_activation_t;
 
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
  * down projection) when the average tokens per expert is small, else
@@ -109,14 +120,22 @@ typedef struct {
   moe_dtype_t dtype;
 } moe_args_t;
 
+/* Per-call options; a zero-initialised struct (or opts == NULL) is the plain
+ * Grok-1 sublayer with automatic kernel choices. */
 typedef struct {
-  moe_gelu_t gelu;            /* MOE_GELU_TANH (default) or MOE_GELU_ERF             */
-  const float* router_bias;   /* [E] fp32 device pointer added to the logits, or NULL */
-  moe_path_t path;            /* kernel family; MOE_PATH_AUTO by default             */
-  int32_t down_splits;        /* WEIGHT_STREAM split-K factor for w_down; 0 = auto    */
-  void* const* stage_events;  /* NULL, or 6 cudaEvent_t (host array) recorded on the
-                                 stream before router, dispatch, gate/up GEMM, down
-                                 GEMM, combine, and after combine (stage timing)     */
+  moe_activation_t activation; /* gate-branch activation, MOE_ACT_GELU_TANH default      */
+  const float* router_bias;    /* [E] fp32 device pointer added to the logits, or NULL    */
+  moe_path_t path;             /* kernel family; MOE_PATH_AUTO by default                */
+  int32_t down_splits;         /* split-K factor for w_down (must divide f/64); 0 = auto  */
+  void* const* stage_events;   /* NULL, or 6 cudaEvent_t (host array) recorded on the
+                                  stream before router, dispatch, gate/up GEMM, down
+                                  GEMM, combine, and after combine (stage timing)        */
+  int32_t renormalize;         /* 0: gates are the softmax probabilities (Grok-1);
+                                  1: gates divided by their sum (Mixtral)                */
+  const void* residual;        /* [T, d] x-dtype device pointer added to the output, or NULL */
+  const float* post_norm_weight; /* [d] fp32 RMSNorm weight applied to the sublayer
+                                  output before the residual add, or NULL (no norm)      */
+  float norm_eps;              /* RMSNorm epsilon (> 0) when post_norm_weight is set      */
 } moe_options_t;
 
 /* Optional outputs for inspection; each is a device pointer or NULL.

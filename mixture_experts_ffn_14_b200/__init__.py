@@ -14,7 +14,7 @@ import ctypes
 
 from . import _native as N
 from ._native import (  # noqa: F401
-    MOE_BF16, MOE_BF16_INT8W, MOE_F32, MOE_GELU_ERF, MOE_GELU_TANH, MOE_PATH_AUTO,
+    MOE_ACT_GELU_ERF, MOE_ACT_GELU_TANH, MOE_ACT_SILU, MOE_BF16, MOE_BF16_INT8W, MOE_F32, MOE_PATH_AUTO,
     MOE_PATH_TOKEN_TILE, MOE_PATH_TOKEN_TILE_SINGLE, MOE_PATH_WEIGHT_STREAM,
 )
 
@@ -92,27 +92,38 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, out, scales=None, stream=None
     return out
 
 
-def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=None, router_bias=None,
-                   gelu=MOE_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, debug=None, stream=None,
-                   stage_events=None, raise_on_error=True):
-    """Forward pass on a caller workspace (a uint8 CUDA tensor). ``debug`` is a
-    dict with any of idx, gates, counts, offsets, perm_token, perm_slot, h.
-    ``stage_events``: 6 torch.cuda.Event (already created, e.g. recorded once)
-    that the library records around its five stages."""
-    T, d = x.shape
-    E, _, f = w_gate.shape
-    sc = _scales(scales)
-    args = N.MoeArgs(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
-                     ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
-                     dtype_code(x, w_gate))
+def _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual, post_norm_weight,
+             norm_eps):
     ev = None
     if stage_events is not None:
         handles = [e.cuda_event for e in stage_events]
         if len(handles) != 6 or not all(handles):
             raise ValueError("moe: stage_events needs 6 created CUDA events")
         ev = (ctypes.c_void_p * 6)(*handles)
-    opts = N.MoeOptions(gelu, _ptr(router_bias), path, down_splits,
-                        ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)) if ev is not None else None)
+    opts = N.MoeOptions(activation, _ptr(router_bias), path, down_splits,
+                        ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)) if ev is not None else None,
+                        int(bool(renormalize)), _ptr(residual), _ptr(post_norm_weight), float(norm_eps))
+    return opts, ev
+
+
+def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=None, router_bias=None,
+                   activation=MOE_ACT_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, debug=None, stream=None,
+                   stage_events=None, renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5,
+                   raise_on_error=True):
+    """Forward pass on a caller workspace (a uint8 CUDA tensor). ``debug`` is a
+    dict with any of idx, gates, counts, offsets, perm_token, perm_slot, h.
+    ``stage_events``: 6 torch.cuda.Event (already created, e.g. recorded once)
+    that the library records around its five stages. ``renormalize``,
+    ``activation``, ``residual``, ``post_norm_weight`` / ``norm_eps``: the
+    moe_options_t variants (Mixtral routing, SiLU, post-RMSNorm + residual)."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    sc = _scales(scales)
+    args = N.MoeArgs(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                     ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
+                     dtype_code(x, w_gate))
+    opts, _keep = _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual,
+                           post_norm_weight, norm_eps)
     dbg = None
     if debug:
         dbg = N.MoeDebug(*[_ptr(debug.get(n)) for n in
@@ -127,7 +138,8 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
 
 
 def moe_forward_noalloc(x, w_router, w_gate, w_up, w_down, out, scales=None, router_bias=None,
-                        gelu=MOE_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, stream=None,
+                        activation=MOE_ACT_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, stream=None,
+                        renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5,
                         raise_on_error=True):
     """Forward pass that allocates no device memory: the library runs it in a
     fixed 32 MiB scratch array of its own, for callers that must not call
@@ -141,7 +153,8 @@ def moe_forward_noalloc(x, w_router, w_gate, w_up, w_down, out, scales=None, rou
     args = N.MoeArgs(_ptr(x), _ptr(w_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                      ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
                      dtype_code(x, w_gate))
-    opts = N.MoeOptions(gelu, _ptr(router_bias), path, down_splits, None)
+    opts, _ = _options(activation, router_bias, path, down_splits, None, renormalize, residual, post_norm_weight,
+                       norm_eps)
     st = N.lib().moe_forward_noalloc(ctypes.byref(args), ctypes.byref(opts), _stream(stream))
     if st != N.MOE_OK and raise_on_error:
         raise MoeError(st, "moe_forward_noalloc")

@@ -9,14 +9,14 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_char_p, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 3
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK = 4, 5, 6
 MOE_F32, MOE_BF16, MOE_BF16_INT8W = 0, 1, 2
-MOE_GELU_TANH, MOE_GELU_ERF = 0, 1
+MOE_ACT_GELU_TANH, MOE_ACT_GELU_ERF, MOE_ACT_SILU = 0, 1, 2
 MOE_PATH_AUTO, MOE_PATH_TOKEN_TILE, MOE_PATH_WEIGHT_STREAM, MOE_PATH_TOKEN_TILE_SINGLE = 0, 1, 2, 3
 
 # Every function include/moe.h exports, with (restype, argtypes).
@@ -35,8 +35,9 @@ class MoeArgs(ctypes.Structure):
 
 
 class MoeOptions(ctypes.Structure):
-    _fields_ = [("gelu", c_int), ("router_bias", c_void_p), ("path", c_int), ("down_splits", c_int32),
-                ("stage_events", POINTER(c_void_p))]
+    _fields_ = [("activation", c_int), ("router_bias", c_void_p), ("path", c_int), ("down_splits", c_int32),
+                ("stage_events", POINTER(c_void_p)), ("renormalize", c_int32), ("residual", c_void_p),
+                ("post_norm_weight", c_void_p), ("norm_eps", c_float)]
 
 
 class MoeDebug(ctypes.Structure):

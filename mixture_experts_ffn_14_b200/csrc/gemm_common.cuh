@@ -1,7 +1,7 @@
 // gemm_common.cuh — pieces shared by the single-CTA and the CTA-pair grouped
 // expert GEMM kernels: tile constants, parameters, the device-side tile
-// scheduler data, GELU, the exact int8 -> bf16 conversion and the token-tile
-// epilogue (GELU(gate) * up -> bf16 H, or gate * down -> fp32 Y).
+// scheduler data, the gate activation, the exact int8 -> bf16 conversion and the token-tile
+// epilogue (act(gate) * up -> bf16 H, or gate * down -> fp32 Y).
 #pragma once
 
 #include <cuda.h>
@@ -39,7 +39,7 @@ struct Params {
   int32_t splits;
   int32_t kb_per_split;  // 64-deep K blocks per tile
   int32_t ntile;         // output columns per tile (128 GATEUP, 256 DOWN)
-  int32_t gelu_mode;
+  int32_t act;           // moe_activation_t of the gate branch
   int32_t select;        // kRunAlways, or run only if the pair / single form is preferred
   int32_t sm_count;      // SMs of the device (same value for both token-tile kernels)
   uint32_t* status;
@@ -128,8 +128,11 @@ __device__ __forceinline__ float tanh_hw(float x) {
   return y;
 }
 
-__device__ __forceinline__ float gelu_f32(float z, int mode) {
-  if (mode == MOE_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+// Gate-branch activation: GELU (tanh form or erf form) or SiLU, the latter as
+// z * sigmoid(z) = 0.5 z (1 + tanh(z / 2)).
+__device__ __forceinline__ float act_f32(float z, int mode) {
+  if (mode == MOE_ACT_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  if (mode == MOE_ACT_SILU) return 0.5f * z * (1.0f + tanh_hw(0.5f * z));
   const float u = 0.7978845608028654f * (z + 0.044715f * z * z * z);
   return 0.5f * z * (1.0f + tanh_hw(u));
 }
@@ -204,7 +207,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
           u0 *= __bfloat162float(p.s1[sc]);
           u1 *= __bfloat162float(p.s1[sc + 1]);
         }
-        packed[j / 2] = pack_bf16x2(gelu_f32(g0, p.gelu_mode) * u0, gelu_f32(g1, p.gelu_mode) * u1);
+        packed[j / 2] = pack_bf16x2(act_f32(g0, p.act) * u0, act_f32(g1, p.act) * u1);
       }
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);

@@ -38,12 +38,13 @@ __device__ __forceinline__ void load_sched(F32Sched& s, const int32_t* counts, c
   __syncthreads();
 }
 
-__device__ __forceinline__ float gelu_ref(float z, int mode) {
-  if (mode == MOE_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+__device__ __forceinline__ float act_ref(float z, int mode) {
+  if (mode == MOE_ACT_GELU_ERF) return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  if (mode == MOE_ACT_SILU) return z / (1.0f + expf(-z));
   return 0.5f * z * (1.0f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)));
 }
 
-// DUAL = true: acc0 = X.B0, acc1 = X.B1, out = GELU(acc0) * acc1   (gate/up)
+// DUAL = true: acc0 = X.B0, acc1 = X.B1, out = act(acc0) * acc1    (gate/up)
 // DUAL = false: out = rowscale[r] * X.B0                            (down)
 template <bool DUAL>
 __global__ void __launch_bounds__(256) moe_f32_expert_gemm(const float* __restrict__ X, const float* __restrict__ B0,
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(256) moe_f32_expert_gemm(const float* __restri
                                                            const int32_t* __restrict__ counts,
                                                            const int32_t* __restrict__ offsets,
                                                            const float* __restrict__ rowscale, int K, int N,
-                                                           int gelu_mode, float* __restrict__ out) {
+                                                           int act, float* __restrict__ out) {
   __shared__ F32Sched sched;
   __shared__ float As[TK][TM];
   __shared__ float Bs0[TK][TN];
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(256) moe_f32_expert_gemm(const float* __restri
       float o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        o[j] = DUAL ? gelu_ref(acc0[i][j], gelu_mode) * acc1[i][j] : acc0[i][j] * rowscale[row];
+        o[j] = DUAL ? act_ref(acc0[i][j], act) * acc1[i][j] : acc0[i][j] * rowscale[row];
       *reinterpret_cast<float4*>(out + row * N + n0 + tx * 4) = make_float4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -138,10 +139,10 @@ int f32_grid(int64_t T, int64_t N) {
 }  // namespace
 
 cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,
-                              const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t gelu_mode,
+                              const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t act,
                               float* h, cudaStream_t s) {
   moe_f32_expert_gemm<true><<<f32_grid(T, f), 256, 0, s>>>(xp, wg, wu, counts, offsets, nullptr,
-                                                          static_cast<int>(d), static_cast<int>(f), gelu_mode, h);
+                                                          static_cast<int>(d), static_cast<int>(f), act, h);
   return cudaGetLastError();
 }
 

@@ -1,7 +1,7 @@
 // gemm_sm100.cu — grouped expert GEMMs on the 5th-generation tensor cores.
 //
 // Two kernels share one persistent, warp-specialised pipeline:
-//   GATEUP: H[r, n] = GELU(Xp[r,:] . Wg[e][:, n]) * (Xp[r,:] . Wu[e][:, n])     (bf16 out)
+//   GATEUP: H[r, n] = act(Xp[r,:] . Wg[e][:, n]) * (Xp[r,:] . Wu[e][:, n])     (bf16 out)
 //   DOWN:   Y[s, r, n] = gate[r] * (H[r, kslice_s] . Wd[e][kslice_s, n])         (fp32 out)
 // for every permuted row r of expert e (rows are expert-contiguous after the
 // dispatch stage). This is the GeGLU expert of the Grok-1 MoE sublayer (Grok-1
@@ -10,7 +10,7 @@
 // Roles per CTA (one CTA per SM, persistent over a static tile list):
 //   warp 0      TMA producer: activation tile + weight tile per 64-deep K stage
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one thread)
-//   warps 4..7  epilogue: tcgen05.ld from TMEM, GELU / gate / scale, global stores
+//   warps 4..7  epilogue: tcgen05.ld from TMEM, activation / gate / scale, global stores
 //   warps 8..15 (int8 weights only) convert the int8 stage to bf16 in shared memory
 //               (two warps per SM sub-partition, so one hides the other's latency)
 //
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (c + j < t.rows) {
-                const float h = gelu_f32(__uint_as_float(g[j]) * sg, p.gelu_mode) * (__uint_as_float(u[j]) * su);
+                const float h = act_f32(__uint_as_float(g[j]) * sg, p.act) * (__uint_as_float(u[j]) * su);
                 hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] = __float2bfloat16_rn(h);
               }
             }
@@ -390,7 +390,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.splits = KIND == DOWN ? a.splits : 1;
   p.kb_per_split = a.K / BK / p.splits;
   p.ntile = KIND == GATEUP ? 128 : 256;
-  p.gelu_mode = a.gelu_mode;
+  p.act = a.act;
   p.select = a.select;
   p.sm_count = device_sm_count();
   p.status = a.status;

@@ -362,7 +362,7 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   p.splits = KIND == DOWN ? a.splits : 1;
   p.kb_per_split = a.K / BK / p.splits;
   p.ntile = KIND == GATEUP ? 128 : 256;
-  p.gelu_mode = a.gelu_mode;
+  p.act = a.act;
   p.select = a.select;
   p.sm_count = device_sm_count();
   p.status = a.status;

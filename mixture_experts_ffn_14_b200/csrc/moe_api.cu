@@ -227,9 +227,13 @@ namespace {
 
 moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_debug_t* dbg, void* workspace,
                          size_t ws_bytes, cudaStream_t stream) {
-  const moe_options_t defaults{MOE_GELU_TANH, nullptr, MOE_PATH_AUTO, 0, nullptr};
+  const moe_options_t defaults{};
   if (!o) o = &defaults;
-  if (o->gelu != MOE_GELU_TANH && o->gelu != MOE_GELU_ERF) return MOE_ERR_INVALID_ARG;
+  if (o->activation < MOE_ACT_GELU_TANH || o->activation > MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
+  if (o->renormalize != 0 && o->renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (o->post_norm_weight && !(o->norm_eps > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if ((o->post_norm_weight && !aligned16(o->post_norm_weight)) || (o->residual && !aligned16(o->residual)))
+    return MOE_ERR_MISALIGNED;
   if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE) return MOE_ERR_INVALID_ARG;
   if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
   if (o->router_bias && !aligned16(o->router_bias)) return MOE_ERR_MISALIGNED;
@@ -266,14 +270,15 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   };
   MOE_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
   MOE_TRY(mark(0));
-  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, idx, gates, hist, stream));
+  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, idx, gates, hist,
+                        stream));
   MOE_TRY(mark(1));
   MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
                           slot_pos, gate_perm, xp, stream));
   MOE_TRY(mark(2));
   if (a->dtype == MOE_F32) {
     MOE_TRY(launch_f32_gateup(static_cast<const float*>(xp), static_cast<const float*>(a->w_gate),
-                              static_cast<const float*>(a->w_up), counts, offsets, T, d, f, o->gelu,
+                              static_cast<const float*>(a->w_up), counts, offsets, T, d, f, o->activation,
                               static_cast<float*>(h), stream));
     MOE_TRY(mark(3));
     MOE_TRY(launch_f32_down(static_cast<const float*>(h), static_cast<const float*>(a->w_down), counts, offsets,
@@ -294,7 +299,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.K = static_cast<int32_t>(d);
     g.N = static_cast<int32_t>(f);
     g.splits = 1;
-    g.gelu_mode = o->gelu;
+    g.act = o->activation;
     g.int8_weights = w8;
     g.weight_stream = L.weight_stream;
     g.status = status;
@@ -334,7 +339,8 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     MOE_TRY(launch_gemm(g2, true));
   }
   MOE_TRY(mark(4));
-  MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, a->out, stream));
+  MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, o->residual, o->post_norm_weight,
+                         o->norm_eps, a->out, stream));
   MOE_TRY(mark(5));
 
   if (dbg) {
@@ -501,7 +507,7 @@ extern "C" moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_op
                                             moe_stream_t stream) {
   const moe_status_t st = check_args(args);
   if (st != MOE_OK || args->T == 0) return st;
-  moe_options_t o{MOE_GELU_TANH, nullptr, MOE_PATH_AUTO, 0, nullptr};
+  moe_options_t o{};
   if (opts) o = *opts;
   if (o.down_splits < 0) return MOE_ERR_INVALID_ARG;
   WorkspaceLayout L = plan_workspace(args->T, args->d, args->f, args->dtype, o.path, o.down_splits, false);

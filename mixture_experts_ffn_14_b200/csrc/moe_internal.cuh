@@ -45,19 +45,22 @@ int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested);
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 
 cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
-                          int64_t d, int32_t* idx, float* gates, int32_t* hist, cudaStream_t s);
+                          int64_t d, int32_t renormalize, int32_t* idx, float* gates, int32_t* hist,
+                          cudaStream_t s);
 
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
                             float* gate_perm, void* xp, cudaStream_t s);
 
+// out[t] = residual[t] + norm(y0 + y1); residual and norm_weight may be NULL.
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
-                           const int32_t* slot_pos, int64_t T, int64_t d, void* out, cudaStream_t s);
+                           const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
+                           const float* norm_weight, float norm_eps, void* out, cudaStream_t s);
 
 // fp32 (SIMT) grouped expert GEMMs.
 cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,
-                              const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t gelu_mode,
+                              const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t act,
                               float* h, cudaStream_t s);
 cudaError_t launch_f32_down(const float* h, const float* wd, const int32_t* counts, const int32_t* offsets,
                             const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, cudaStream_t s);
@@ -76,7 +79,7 @@ struct TcGemmArgs {
   int64_t rows;             // 2T
   int32_t K, N;
   int32_t splits;           // DOWN split-K factor (1 for GATEUP)
-  int32_t gelu_mode;
+  int32_t act;              // moe_activation_t
   bool int8_weights;
   bool weight_stream;
   int32_t select;           // 0: always run; 1 / 2: run only if the pair / single token-tile form is preferred

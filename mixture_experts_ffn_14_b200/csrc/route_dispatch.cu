@@ -8,7 +8,9 @@
 //              order; integer and deterministic (no capacity, no drop: ch. 10,
 //              section 10.3.2)
 //   combine  : out[t] = (gate-weighted slot-0 rows) + (slot-1 rows), summing the
-//              split-K partials in a fixed order; no atomics on the output.
+//              split-K partials in a fixed order; no atomics on the output;
+//              optionally followed by the post-RMSNorm and the residual add
+//              (sandwich norm: ch. 10, section 10.3.1)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -67,7 +69,8 @@ template <typename TX>
 __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const TX* __restrict__ x,
                                                                      const float* __restrict__ wr,
                                                                      const float* __restrict__ bias, int64_t T,
-                                                                     int64_t d, int32_t* __restrict__ idx,
+                                                                     int64_t d, int32_t renormalize,
+                                                                     int32_t* __restrict__ idx,
                                                                      float* __restrict__ gates,
                                                                      int32_t* __restrict__ hist) {
   constexpr int V = Vec<TX>::N;
@@ -131,8 +134,14 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const TX* __
       for (int e = 0; e < kE; ++e) s += expf(l[e] - m);
       idx[2 * t] = e0;
       idx[2 * t + 1] = e1;
-      gates[2 * t] = 1.0f / s;
-      gates[2 * t + 1] = expf(l[e1] - m) / s;
+      const float p1 = expf(l[e1] - m);
+      if (renormalize) {  // Mixtral: the two probabilities divided by their sum
+        gates[2 * t] = 1.0f / (1.0f + p1);
+        gates[2 * t + 1] = p1 / (1.0f + p1);
+      } else {
+        gates[2 * t] = 1.0f / s;
+        gates[2 * t + 1] = p1 / s;
+      }
       atomicAdd(&cnt[e0], 1);
       atomicAdd(&cnt[e1], 1);
     }
@@ -285,17 +294,89 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
   }
 }
 
+template <typename TO>
+__device__ __forceinline__ float4 load4(const TO* p);
+
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+// Combine with the sublayer's post-RMSNorm and/or residual add: one CTA per
+// token row. Pass 1 forms y = (slot-0 rows) + (slot-1 rows) in fp32 and its sum
+// of squares (fixed reduction order: per-thread strided sums, then a fixed
+// tree); pass 2 forms y again (its rows are now in L2) and writes
+// residual + w * y * rsqrt(mean(y^2) + eps).
+template <typename TO>
+__global__ void __launch_bounds__(256) moe_combine_norm_kernel(const float* __restrict__ y, int64_t split_stride,
+                                                               int32_t splits, const int32_t* __restrict__ slot_pos,
+                                                               int64_t d, const TO* __restrict__ residual,
+                                                               const float* __restrict__ norm_weight, float eps,
+                                                               TO* __restrict__ out) {
+  __shared__ float red[8];
+  const int64_t t = blockIdx.x;
+  const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
+  auto row_y = [&](int64_t c) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int s = 0; s < splits; ++s) {
+      const float4 u = *reinterpret_cast<const float4*>(y + s * split_stride + p0 * d + c);
+      const float4 v = *reinterpret_cast<const float4*>(y + s * split_stride + p1 * d + c);
+      a.x += u.x; a.y += u.y; a.z += u.z; a.w += u.w;
+      b.x += v.x; b.y += v.y; b.z += v.z; b.w += v.w;
+    }
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+  };
+  float scale = 1.0f;
+  if (norm_weight) {
+    float ss = 0.0f;
+    for (int64_t c = 4 * threadIdx.x; c < d; c += 4 * blockDim.x) {
+      const float4 v = row_y(c);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float v = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.0f;
+      v = warp_sum(v);
+      if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  }
+  for (int64_t c = 4 * threadIdx.x; c < d; c += 4 * blockDim.x) {
+    float4 v = row_y(c);
+    if (norm_weight) {
+      const float4 w = *reinterpret_cast<const float4*>(norm_weight + c);
+      v = make_float4(v.x * scale * w.x, v.y * scale * w.y, v.z * scale * w.z, v.w * scale * w.w);
+    }
+    if (residual) {
+      const float4 r = load4<TO>(residual + t * d + c);
+      v = make_float4(v.x + r.x, v.y + r.y, v.z + r.z, v.w + r.w);
+    }
+    store4<TO>(out + t * d + c, v);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
-                          int64_t d, int32_t* idx, float* gates, int32_t* hist, cudaStream_t s) {
+                          int64_t d, int32_t renormalize, int32_t* idx, float* gates, int32_t* hist,
+                          cudaStream_t s) {
   const int64_t nblk = (T + kRouteTokens - 1) / kRouteTokens;
   if (dtype == MOE_F32)
     moe_router_kernel<float><<<static_cast<unsigned>(nblk), kRouterThreads, 0, s>>>(
-        static_cast<const float*>(x), w_router, bias, T, d, idx, gates, hist);
+        static_cast<const float*>(x), w_router, bias, T, d, renormalize, idx, gates, hist);
   else
     moe_router_kernel<__nv_bfloat16><<<static_cast<unsigned>(nblk), kRouterThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, idx, gates, hist);
+        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, hist);
   return cudaGetLastError();
 }
 
@@ -315,7 +396,19 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
 }
 
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
-                           const int32_t* slot_pos, int64_t T, int64_t d, void* out, cudaStream_t s) {
+                           const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
+                           const float* norm_weight, float norm_eps, void* out, cudaStream_t s) {
+  if (residual || norm_weight) {
+    if (dtype == MOE_F32)
+      moe_combine_norm_kernel<float><<<static_cast<unsigned>(T), 256, 0, s>>>(
+          y, split_stride, splits, slot_pos, d, static_cast<const float*>(residual), norm_weight, norm_eps,
+          static_cast<float*>(out));
+    else
+      moe_combine_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, 0, s>>>(
+          y, split_stride, splits, slot_pos, d, static_cast<const __nv_bfloat16*>(residual), norm_weight,
+          norm_eps, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+  }
   const int64_t n = T * (d / 4);
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(device_sm_count()) * 8);
   if (dtype == MOE_F32)

@@ -22,8 +22,8 @@ def np64(t) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, gelu=moe.MOE_GELU_TANH, down_splits=0, want_h=True,
-            stream=None) -> dict:
+def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, activation=moe.MOE_ACT_GELU_TANH, down_splits=0, want_h=True,
+            stream=None, renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5) -> dict:
     """One forward through moe_forward_ex with every debug output requested."""
     x = inp["x"]
     T, d = x.shape
@@ -44,7 +44,9 @@ def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, gelu=moe.MOE_GELU_TANH, down_s
         dbg["h"] = torch.empty((2 * T, f), dtype=x.dtype, device=dev)
     scales = (inp["s_gate"], inp["s_up"], inp["s_down"]) if "s_gate" in inp else None
     moe.moe_forward_ex(x, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws, scales=scales,
-                       router_bias=inp.get("router_bias"), gelu=gelu, path=path, down_splits=down_splits,
+                       router_bias=inp.get("router_bias"), activation=activation, path=path, down_splits=down_splits,
+                       renormalize=renormalize, residual=residual, post_norm_weight=post_norm_weight,
+                       norm_eps=norm_eps,
                        debug=dbg, stream=stream)
     torch.cuda.synchronize()
     st, code = moe.moe_device_status(ws)
@@ -56,7 +58,7 @@ def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, gelu=moe.MOE_GELU_TANH, down_s
     return res
 
 
-def expected_routing(x64, wr64, bias64, gpu_idx) -> tuple:
+def expected_routing(x64, wr64, bias64, gpu_idx, renormalize=False) -> tuple:
     """Oracle routing; near-tie tokens take the GPU's pair only if the oracle
     lists it as valid. Returns (routing dict with idx/gates, n_excluded)."""
     r = oracle.route(x64, wr64, bias64)
@@ -69,6 +71,8 @@ def expected_routing(x64, wr64, bias64, gpu_idx) -> tuple:
         if g in alts:
             idx[t] = g
     gates = np.take_along_axis(r["probs"], idx.astype(np.int64), axis=1)
+    if renormalize:
+        gates = gates / gates.sum(axis=1, keepdims=True)
     return {"idx": idx, "gates": gates, "probs": r["probs"], "logits32": r["logits32"]}, len(amb)
 
 
@@ -114,16 +118,23 @@ def expert_getter(inp: dict):
     return get
 
 
-def full_check(inp: dict, gpu: dict, tokens=None, check_h=True, gelu_mode="tanh"):
-    """Routing + dispatch bit-exact, out (and h) within tolerance on `tokens`."""
+def full_check(inp: dict, gpu: dict, tokens=None, check_h=True, gelu_mode="tanh", renormalize=False,
+               residual=None, post_norm_weight=None, norm_eps=1e-5):
+    """Routing + dispatch bit-exact, out (and h) within tolerance on `tokens`.
+    With residual / post_norm_weight the oracle output is post-normed and added
+    to the residual row by row, as the library's options ask for."""
     o = oracle_inputs(inp)
-    routing, n_amb = expected_routing(o["x"], o["w_router"], o["bias"], gpu["idx"])
+    routing, n_amb = expected_routing(o["x"], o["w_router"], o["bias"], gpu["idx"], renormalize)
     dsp = check_routing_and_dispatch(gpu, routing)
     T = o["x"].shape[0]
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
     res = oracle.forward_sparse(o["x"], o["w_router"], expert_getter(inp), routing=routing, tokens=tok,
                                 return_h=check_h, gelu_mode=gelu_mode)
-    worst = assert_close(gpu["out"][tok], res["out"], "out")
+    ref = res["out"]
+    if residual is not None or post_norm_weight is not None:
+        ref = oracle.post_norm_residual(ref, None if residual is None else np64(residual)[tok],
+                                        None if post_norm_weight is None else np64(post_norm_weight), norm_eps)
+    worst = assert_close(gpu["out"][tok], ref, "out")
     if check_h:
         pos = dsp["slot_pos"][tok]               # [n, 2] permuted rows of each (token, slot)
         h_gpu = np64(gpu["h"][torch.as_tensor(pos.reshape(-1), device=gpu["h"].device)])

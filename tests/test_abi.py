@@ -124,3 +124,17 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError):
         moe.moe_forward(x, torch.zeros(256, 8), w, w, torch.zeros(8, 128, 256, dtype=torch.bfloat16),
                         torch.empty_like(x), stream=0)
+
+
+def test_option_checks():
+    a = _args()
+    bad = N.MoeOptions(3, None, 0, 0, None, 0, None, None, 0.0)      # no such activation
+    assert _call(a, opts=bad) == N.MOE_ERR_INVALID_ARG
+    bad = N.MoeOptions(0, None, 0, 0, None, 2, None, None, 0.0)      # renormalize must be 0 or 1
+    assert _call(a, opts=bad) == N.MOE_ERR_INVALID_ARG
+    bad = N.MoeOptions(0, None, 0, 0, None, 0, None, 0x50000000, 0.0)  # post-norm needs eps > 0
+    assert _call(a, opts=bad) == N.MOE_ERR_INVALID_ARG
+    bad = N.MoeOptions(0, None, 0, 0, None, 0, None, 0x50000004, 1e-5)
+    assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED
+    bad = N.MoeOptions(0, None, 0, 0, None, 0, 0x50000008, None, 0.0)
+    assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED

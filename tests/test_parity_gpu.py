@@ -45,7 +45,7 @@ def test_f32_ragged_token_counts(T):
 
 def test_f32_erf_gelu():
     inp = tiny_f32(seed=9)
-    full_check(inp, run_gpu(inp, gelu=moe.MOE_GELU_ERF), gelu_mode="erf")
+    full_check(inp, run_gpu(inp, activation=moe.MOE_ACT_GELU_ERF), gelu_mode="erf")
 
 
 # ------------------------------------------------------------------ bf16 --
@@ -113,7 +113,7 @@ def test_bf16_skew_bias_workload_small():
 
 def test_bf16_erf_gelu():
     inp = small_bf16(130, seed=14)
-    full_check(inp, run_gpu(inp, gelu=moe.MOE_GELU_ERF), gelu_mode="erf")
+    full_check(inp, run_gpu(inp, activation=moe.MOE_ACT_GELU_ERF), gelu_mode="erf")
 
 
 # ------------------------------------------------------------------ int8 --
@@ -168,3 +168,63 @@ def test_zero_tokens_is_a_noop():
     x0 = inp["x"][:0]
     out = torch.empty((0, inp["x"].shape[1]), dtype=torch.bfloat16, device=DEV)
     moe.moe_forward(x0, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
+
+
+# ------------------------------------------- next rows: Mixtral, post-norm --
+
+VARIANTS = [
+    dict(renormalize=True),
+    dict(activation=moe.MOE_ACT_SILU),
+    dict(renormalize=True, activation=moe.MOE_ACT_SILU),
+    dict(post_norm=True),
+    dict(residual=True),
+    dict(post_norm=True, residual=True, renormalize=True),
+]
+
+
+def _variant_args(inp, v, seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    T, d = inp["x"].shape
+    kw = {k: v[k] for k in ("renormalize", "activation") if k in v}
+    if v.get("residual"):
+        kw["residual"] = torch.randn((T, d), generator=g, device=DEV).to(inp["x"].dtype)
+    if v.get("post_norm"):
+        kw["post_norm_weight"] = (0.5 + torch.rand(d, generator=g, device=DEV)).float()
+        kw["norm_eps"] = 1e-5
+    return kw
+
+
+def _oracle_kw(kw):
+    okw = {k: kw[k] for k in ("renormalize", "residual", "post_norm_weight", "norm_eps") if k in kw}
+    if kw.get("activation") == moe.MOE_ACT_SILU:
+        okw["gelu_mode"] = "silu"
+    return okw
+
+
+@pytest.mark.parametrize("vi", range(len(VARIANTS)))
+def test_variants_f32(vi):
+    inp = tiny_f32(seed=40 + vi)
+    kw = _variant_args(inp, VARIANTS[vi], vi)
+    full_check(inp, run_gpu(inp, **kw), **_oracle_kw(kw))
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("vi", range(len(VARIANTS)))
+def test_variants_bf16(vi, path):
+    inp = small_bf16(300, seed=50 + vi)
+    kw = _variant_args(inp, VARIANTS[vi], vi)
+    full_check(inp, run_gpu(inp, path=path, **kw), **_oracle_kw(kw))
+
+
+@pytest.mark.parametrize("vi", [2, 5])
+def test_variants_int8(vi):
+    inp = small_bf16(200, seed=60 + vi, int8=True)
+    kw = _variant_args(inp, VARIANTS[vi], vi)
+    full_check(inp, run_gpu(inp, **kw), **_oracle_kw(kw))
+
+
+def test_renormalized_gates_sum_to_one():
+    inp = small_bf16(64, seed=70)
+    gpu = run_gpu(inp, renormalize=True, want_h=False)
+    assert np.abs(gpu["gates"].sum(1) - 1.0).max() < 1e-6
