@@ -202,10 +202,13 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
     o = align_up(o + bytes);
     return at;
   };
+  L.router_slices = router_slices(T, d, dtype);
   L.status = take(kAlign);
+  L.arrivals = take(sizeof(int32_t) * L.nblk);  // right after the status word: one memset clears both
   L.idx = take(sizeof(int32_t) * rows);
   L.gates = take(sizeof(float) * rows);
   L.hist = take(sizeof(int32_t) * L.nblk * kE);
+  L.logits_part = L.router_slices > 1 ? take(sizeof(float) * L.router_slices * T * kE) : 0;
   L.counts = take(sizeof(int32_t) * kE);
   L.offsets = take(sizeof(int32_t) * (kE + 1));
   L.perm_token = take(sizeof(int32_t) * rows);
@@ -249,6 +252,8 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
   float* gates = reinterpret_cast<float*>(ws + L.gates);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(ws + L.arrivals);
+  float* logits_part = L.router_slices > 1 ? reinterpret_cast<float*>(ws + L.logits_part) : nullptr;
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
   int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
   int32_t* perm_token = reinterpret_cast<int32_t*>(ws + L.perm_token);
@@ -268,10 +273,11 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   auto mark = [&](int i) {
     return o->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(o->stage_events[i]), stream) : cudaSuccess;
   };
-  MOE_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), stream));
+  // Status word and router arrival counters start at zero.
+  MOE_TRY(cudaMemsetAsync(status, 0, L.arrivals + sizeof(int32_t) * L.nblk - L.status, stream));
   MOE_TRY(mark(0));
-  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, idx, gates, hist,
-                        stream));
+  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, L.router_slices,
+                        logits_part, arrivals, idx, gates, hist, stream));
   MOE_TRY(mark(1));
   MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
                           slot_pos, gate_perm, xp, stream));

@@ -27,10 +27,12 @@ enum : uint32_t {
 
 // Byte offsets of the regions of one call's workspace (each 256-aligned).
 struct WorkspaceLayout {
-  size_t status, idx, gates, hist, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm;
+  size_t status, arrivals, idx, gates, hist, logits_part, counts, offsets, perm_token, perm_slot, slot_pos,
+      gate_perm;
   size_t xp, h, y, total;
   int64_t nblk;      // router / dispatch CTAs
   int32_t splits;    // split-K factor of the down projection
+  int32_t router_slices;  // d slices of the router grid
   bool weight_stream;
 };
 
@@ -44,9 +46,13 @@ int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested);
 
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 
+// Router: grid of (token blocks, d slices). With slices > 1 the CTAs store
+// partial logits in `partial` [slices, T, E] and count their arrivals per token
+// block in `arrivals` [nblk] (zero on entry); the last one finishes the block.
+int32_t router_slices(int64_t T, int64_t d, moe_dtype_t dtype);
 cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
-                          int64_t d, int32_t renormalize, int32_t* idx, float* gates, int32_t* hist,
-                          cudaStream_t s);
+                          int64_t d, int32_t renormalize, int32_t slices, float* partial, int32_t* arrivals,
+                          int32_t* idx, float* gates, int32_t* hist, cudaStream_t s);
 
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,

@@ -24,6 +24,7 @@ namespace {
 
 constexpr int kRouterThreads = 256;
 constexpr int kTokPerWarp = kRouteTokens / (kRouterThreads / 32);  // 4
+constexpr int kWrRows = 1024;  // router-weight rows staged in shared memory at a time
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -63,47 +64,104 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
-// One CTA = 32 tokens, one warp = 4 tokens; lanes split the hidden dimension in
-// 16-byte vectors. Writes idx/gates per token and the CTA's per-expert slot count.
+// Top-2 of the 8 logits (strict comparisons keep the lower index on ties),
+// softmax in fp32 and the gates (optionally renormalised), for token t.
+__device__ __forceinline__ void finalize_token(const float (&l)[kE], int64_t t, int32_t renormalize,
+                                               int32_t* __restrict__ idx, float* __restrict__ gates, int* cnt) {
+  int e0 = 0;
+  float m = l[0];
+#pragma unroll
+  for (int e = 1; e < kE; ++e)
+    if (l[e] > m) {
+      e0 = e;
+      m = l[e];
+    }
+  int e1 = -1;
+  float m1 = 0.0f;
+#pragma unroll
+  for (int e = 0; e < kE; ++e)
+    if (e != e0 && (e1 < 0 || l[e] > m1)) {
+      e1 = e;
+      m1 = l[e];
+    }
+  float s = 0.0f;
+#pragma unroll
+  for (int e = 0; e < kE; ++e) s += expf(l[e] - m);
+  idx[2 * t] = e0;
+  idx[2 * t + 1] = e1;
+  const float p1 = expf(m1 - m);
+  if (renormalize) {  // Mixtral: the two probabilities divided by their sum
+    gates[2 * t] = 1.0f / (1.0f + p1);
+    gates[2 * t + 1] = p1 / (1.0f + p1);
+  } else {
+    gates[2 * t] = 1.0f / s;
+    gates[2 * t + 1] = p1 / s;
+  }
+  atomicAdd(&cnt[e0], 1);
+  atomicAdd(&cnt[e1], 1);
+}
+
+// Grid (token blocks of 32, d slices). One warp = 4 tokens; lanes split the CTA's
+// slice of the hidden dimension in 16-byte vectors, the four tokens' loads
+// issued together. With one slice the CTA finishes its tokens from registers.
+// With several, each CTA stores its partial logits; the CTA that finds itself
+// last for its token block (atomic counter, no waiting) sums the partials in
+// slice order (so the result does not depend on arrival order) and finishes.
+// Writes idx/gates per token and the block's per-expert slot count.
 template <typename TX>
-__global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const TX* __restrict__ x,
-                                                                     const float* __restrict__ wr,
-                                                                     const float* __restrict__ bias, int64_t T,
-                                                                     int64_t d, int32_t renormalize,
-                                                                     int32_t* __restrict__ idx,
-                                                                     float* __restrict__ gates,
-                                                                     int32_t* __restrict__ hist) {
+__global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(
+    const TX* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ bias, int64_t T, int64_t d,
+    int32_t renormalize, int32_t slices, float* __restrict__ partial, int32_t* __restrict__ arrivals,
+    int32_t* __restrict__ idx, float* __restrict__ gates, int32_t* __restrict__ hist) {
   constexpr int V = Vec<TX>::N;
   __shared__ int cnt[kE];
+  __shared__ int last;
+  __shared__ float4 wsm[(kWrRows * kE + (kWrRows / 4) * 4) / 4];
   if (threadIdx.x < kE) cnt[threadIdx.x] = 0;
   __syncthreads();
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokens + warp * kTokPerWarp;
+  const int64_t blk = blockIdx.x;
+  const int64_t t0 = blk * kRouteTokens + warp * kTokPerWarp;
+  const int64_t len = d / slices;
+  const int64_t c_begin = static_cast<int64_t>(blockIdx.y) * len;
+  const TX* rows[kTokPerWarp];
+#pragma unroll
+  for (int j = 0; j < kTokPerWarp; ++j) rows[j] = x + min(t0 + j, T - 1) * d;  // clamped: always in bounds
   float acc[kTokPerWarp][kE];
 #pragma unroll
   for (int j = 0; j < kTokPerWarp; ++j)
 #pragma unroll
     for (int e = 0; e < kE; ++e) acc[j][e] = 0.0f;
 
-  for (int64_t c = static_cast<int64_t>(lane) * V; c < d; c += 32 * V) {
-    float w[V][kE];
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-      const float4 a = *reinterpret_cast<const float4*>(wr + (c + i) * kE);
-      const float4 b = *reinterpret_cast<const float4*>(wr + (c + i) * kE + 4);
-      w[i][0] = a.x; w[i][1] = a.y; w[i][2] = a.z; w[i][3] = a.w;
-      w[i][4] = b.x; w[i][5] = b.y; w[i][6] = b.z; w[i][7] = b.w;
+  // The slice's router weights pass through shared memory in chunks of
+  // kWrRows rows, loaded with coalesced 16-byte reads. A lane then needs rows
+  // base + V*lane + i: in global memory those sit 32*V bytes apart per lane (one
+  // sector per lane per load); in shared memory each group of V rows is followed
+  // by 16 bytes of padding, which spreads the lanes' 16-byte reads over all banks.
+  for (int64_t cc = c_begin; cc < c_begin + len; cc += kWrRows) {
+    const int rows_here = static_cast<int>(min(static_cast<int64_t>(kWrRows), c_begin + len - cc));
+    __syncthreads();
+    for (int q = threadIdx.x; q < rows_here * 2; q += blockDim.x) {
+      const int r = q >> 1;
+      wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] = *reinterpret_cast<const float4*>(wr + (cc + r) * kE + (q & 1) * 4);
     }
+    __syncthreads();
+#pragma unroll 2
+    for (int r0 = lane * V; r0 < rows_here; r0 += 32 * V) {
+      float xv[kTokPerWarp][V];
 #pragma unroll
-    for (int j = 0; j < kTokPerWarp; ++j) {
-      if (t0 + j < T) {
-        float xv[V];
-        Vec<TX>::load(x + (t0 + j) * d + c, xv);
+      for (int j = 0; j < kTokPerWarp; ++j) Vec<TX>::load(rows[j] + cc + r0, xv[j]);
 #pragma unroll
-        for (int i = 0; i < V; ++i)
+      for (int i = 0; i < V; ++i) {
+        const int r = r0 + i;
+        const float4 a = wsm[(r * kE + (r / V) * 4) / 4];
+        const float4 b = wsm[(r * kE + (r / V) * 4) / 4 + 1];
+        const float w[kE] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-          for (int e = 0; e < kE; ++e) acc[j][e] = fmaf(xv[i], w[i][e], acc[j][e]);
+        for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+          for (int e = 0; e < kE; ++e) acc[j][e] = fmaf(xv[j][i], w[e], acc[j][e]);
       }
     }
   }
@@ -112,42 +170,53 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const TX* __
 #pragma unroll
     for (int e = 0; e < kE; ++e) acc[j][e] = warp_sum(acc[j][e]);
 
+  if (slices == 1) {
 #pragma unroll
-  for (int j = 0; j < kTokPerWarp; ++j) {
-    const int64_t t = t0 + j;
-    if (lane == j && t < T) {
+    for (int j = 0; j < kTokPerWarp; ++j) {
+      if (lane == j && t0 + j < T) {
+        float l[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) l[e] = acc[j][e] + (bias ? bias[e] : 0.0f);
+        finalize_token(l, t0 + j, renormalize, idx, gates, cnt);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kTokPerWarp; ++j) {
+      if (lane == j && t0 + j < T) {
+        float* dst = partial + (static_cast<int64_t>(blockIdx.y) * T + t0 + j) * kE;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&arrivals[blk], 1) == slices - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int64_t t = blk * kRouteTokens + threadIdx.x;
+    if (threadIdx.x < kRouteTokens && t < T) {
       float l[kE];
 #pragma unroll
-      for (int e = 0; e < kE; ++e) l[e] = acc[j][e] + (bias ? bias[e] : 0.0f);
-      // Top-2 by value; strict comparisons keep the lower index on ties.
-      int e0 = 0;
+      for (int e = 0; e < kE; ++e) l[e] = bias ? bias[e] : 0.0f;
+      float sum[kE];
 #pragma unroll
-      for (int e = 1; e < kE; ++e)
-        if (l[e] > l[e0]) e0 = e;
-      int e1 = e0 == 0 ? 1 : 0;
-#pragma unroll
-      for (int e = 0; e < kE; ++e)
-        if (e != e0 && l[e] > l[e1]) e1 = e;
-      const float m = l[e0];
-      float s = 0.0f;
-#pragma unroll
-      for (int e = 0; e < kE; ++e) s += expf(l[e] - m);
-      idx[2 * t] = e0;
-      idx[2 * t + 1] = e1;
-      const float p1 = expf(l[e1] - m);
-      if (renormalize) {  // Mixtral: the two probabilities divided by their sum
-        gates[2 * t] = 1.0f / (1.0f + p1);
-        gates[2 * t + 1] = p1 / (1.0f + p1);
-      } else {
-        gates[2 * t] = 1.0f / s;
-        gates[2 * t + 1] = p1 / s;
+      for (int e = 0; e < kE; ++e) sum[e] = 0.0f;
+      for (int sl = 0; sl < slices; ++sl) {
+        const float* src = partial + (static_cast<int64_t>(sl) * T + t) * kE;
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(src));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + 4));
+        sum[0] += a.x; sum[1] += a.y; sum[2] += a.z; sum[3] += a.w;
+        sum[4] += b.x; sum[5] += b.y; sum[6] += b.z; sum[7] += b.w;
       }
-      atomicAdd(&cnt[e0], 1);
-      atomicAdd(&cnt[e1], 1);
+#pragma unroll
+      for (int e = 0; e < kE; ++e) l[e] += sum[e];
+      finalize_token(l, t, renormalize, idx, gates, cnt);
     }
   }
   __syncthreads();
-  if (threadIdx.x < kE) hist[static_cast<int64_t>(blockIdx.x) * kE + threadIdx.x] = cnt[threadIdx.x];
+  if (threadIdx.x < kE) hist[blk * kE + threadIdx.x] = cnt[threadIdx.x];
 }
 
 // Same 32-token range per CTA as the router. Each CTA sums the per-CTA
@@ -160,6 +229,8 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     const float* __restrict__ gates, const int32_t* __restrict__ hist, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
     int32_t* __restrict__ slot_pos, float* __restrict__ gate_perm, TX* __restrict__ xp) {
+  // blockIdx.y splits the row gather of the block across gridDim.y CTAs; all of
+  // them rank the block's tokens (cheap), the first one writes the permutation.
   __shared__ int red[8][2 * kE];
   __shared__ int base[kE];
   __shared__ int pos_sm[kRouteTokens][2];
@@ -202,13 +273,13 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     int off = 0;
     for (int e = 0; e < kE; ++e) {
       base[e] = off + before[e];
-      if (blk == 0) {
+      if (blk == 0 && blockIdx.y == 0) {
         counts[e] = total[e];
         offsets[e] = off;
       }
       off += total[e];
     }
-    if (blk == 0) offsets[kE] = off;
+    if (blk == 0 && blockIdx.y == 0) offsets[kE] = off;
   }
   __syncthreads();
 
@@ -226,7 +297,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
       if (a == e) pa = r;
       if (b == e) pb = r;
     }
-    if (valid) {
+    if (valid && blockIdx.y == 0) {
       perm_token[pa] = static_cast<int32_t>(t);
       perm_slot[pa] = 0;
       perm_token[pb] = static_cast<int32_t>(t);
@@ -241,16 +312,33 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
   }
   __syncthreads();
 
-  // Gather: 64 rows of d elements, as 16-byte vectors.
+  // Gather: 64 rows of d elements, as 16-byte vectors; eight loads in flight
+  // per thread before their stores.
   const int64_t vec_per_row = d * static_cast<int64_t>(sizeof(TX)) / 16;
   const uint4* src = reinterpret_cast<const uint4*>(x);
   uint4* dst = reinterpret_cast<uint4*>(xp);
-  for (int64_t i = threadIdx.x; i < 2 * kRouteTokens * vec_per_row; i += blockDim.x) {
-    const int r = static_cast<int>(i / vec_per_row);
-    const int64_t c = i - r * vec_per_row;
-    const int tl = r >> 1, s = r & 1;
-    const int pos = pos_sm[tl][s];
-    if (pos >= 0) dst[static_cast<int64_t>(pos) * vec_per_row + c] = src[(blk * kRouteTokens + tl) * vec_per_row + c];
+  const int64_t total = 2 * kRouteTokens * vec_per_row;
+  const int64_t stride = static_cast<int64_t>(blockDim.x) * gridDim.y;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; i0 < total; i0 += 8 * stride) {
+    uint4 v[8];
+    int64_t o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t i = i0 + u * stride;
+      o[u] = -1;
+      if (i < total) {
+        const int r = static_cast<int>(i / vec_per_row);
+        const int64_t c = i - r * vec_per_row;
+        const int pos = pos_sm[r >> 1][r & 1];
+        if (pos >= 0) {
+          v[u] = src[(blk * kRouteTokens + (r >> 1)) * vec_per_row + c];
+          o[u] = static_cast<int64_t>(pos) * vec_per_row + c;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (o[u] >= 0) dst[o[u]] = v[u];
   }
 }
 
@@ -278,19 +366,36 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
                                                           int64_t T, int64_t d, TO* __restrict__ out) {
   const int64_t q = d / 4;
   const int64_t n = T * q;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / q;
-    const int64_t c = (i - t * q) * 4;
-    const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    for (int s = 0; s < splits; ++s) {
-      const float4 u = *reinterpret_cast<const float4*>(y + s * split_stride + p0 * d + c);
-      const float4 v = *reinterpret_cast<const float4*>(y + s * split_stride + p1 * d + c);
-      a.x += u.x; a.y += u.y; a.z += u.z; a.w += u.w;
-      b.x += v.x; b.y += v.y; b.z += v.z; b.w += v.w;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // Four outputs per thread per pass, their loads issued before any store.
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n; i0 += 4 * stride) {
+    float4 r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      r[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < n) {
+        const int64_t t = i / q;
+        const int64_t c = (i - t * q) * 4;
+        const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        for (int s = 0; s < splits; ++s) {
+          const float4 uu = *reinterpret_cast<const float4*>(y + s * split_stride + p0 * d + c);
+          const float4 vv = *reinterpret_cast<const float4*>(y + s * split_stride + p1 * d + c);
+          a.x += uu.x; a.y += uu.y; a.z += uu.z; a.w += uu.w;
+          b.x += vv.x; b.y += vv.y; b.z += vv.z; b.w += vv.w;
+        }
+        r[u] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+      }
     }
-    store4<TO>(out + t * d + c, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < n) {
+        const int64_t t = i / q;
+        store4<TO>(out + t * d + (i - t * q) * 4, r[u]);
+      }
+    }
   }
 }
 
@@ -367,16 +472,30 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(const float* __re
 
 }  // namespace
 
-cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
-                          int64_t d, int32_t renormalize, int32_t* idx, float* gates, int32_t* hist,
-                          cudaStream_t s) {
+int32_t router_slices(int64_t T, int64_t d, moe_dtype_t dtype) {
+  // Split d so that about two CTAs per SM run; each slice a whole number of
+  // 32-lane x 16-byte steps.
+  const int64_t chunk = 32 * (dtype == MOE_F32 ? 4 : 8);
+  const int64_t nchunks = d / chunk;
   const int64_t nblk = (T + kRouteTokens - 1) / kRouteTokens;
+  int64_t s = std::min<int64_t>(nchunks, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk));
+  while (s > 1 && nchunks % s != 0) --s;
+  return static_cast<int32_t>(std::max<int64_t>(1, s));
+}
+
+cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias, int64_t T,
+                          int64_t d, int32_t renormalize, int32_t slices, float* partial, int32_t* arrivals,
+                          int32_t* idx, float* gates, int32_t* hist, cudaStream_t s) {
+  const int64_t nblk = (T + kRouteTokens - 1) / kRouteTokens;
+  const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(slices), 1);
   if (dtype == MOE_F32)
-    moe_router_kernel<float><<<static_cast<unsigned>(nblk), kRouterThreads, 0, s>>>(
-        static_cast<const float*>(x), w_router, bias, T, d, renormalize, idx, gates, hist);
+    moe_router_kernel<float><<<grid, kRouterThreads, 0, s>>>(static_cast<const float*>(x), w_router, bias, T, d,
+                                                             renormalize, slices, partial, arrivals, idx, gates,
+                                                             hist);
   else
-    moe_router_kernel<__nv_bfloat16><<<static_cast<unsigned>(nblk), kRouterThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, hist);
+    moe_router_kernel<__nv_bfloat16><<<grid, kRouterThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, slices, partial, arrivals, idx,
+        gates, hist);
   return cudaGetLastError();
 }
 
@@ -384,12 +503,14 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
                             float* gate_perm, void* xp, cudaStream_t s) {
+  const int64_t g = std::min<int64_t>(16, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk));
+  const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(g), 1);
   if (dtype == MOE_F32)
-    moe_dispatch_kernel<float><<<static_cast<unsigned>(nblk), 256, 0, s>>>(
+    moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(
         static_cast<const float*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
         slot_pos, gate_perm, static_cast<float*>(xp));
   else
-    moe_dispatch_kernel<__nv_bfloat16><<<static_cast<unsigned>(nblk), 256, 0, s>>>(
+    moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
         perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp));
   return cudaGetLastError();
