@@ -233,6 +233,8 @@ def timed_steps(run, x, out, K, flush, clk=None):
 
 
 def max_over_ranks(v, dist, dev):
+    """Largest value over the ranks (the slowest replica's time). `dev` is the
+    device the reduction runs on: a CUDA device under NCCL, the CPU under gloo."""
     if dist is None:
         return v
     import torch
@@ -240,6 +242,20 @@ def max_over_ranks(v, dist, dev):
     t = torch.tensor([v], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, steps, work_per_step, t_max_ms):
+    """Whole-job rate: every rank did `steps` steps of `work_per_step` units,
+    the job took as long as its slowest rank."""
+    return world * steps * work_per_step / (t_max_ms / 1e3)
+
+
+def launches_per_step(wl, path):
+    """Kernels of ours per step: router, dispatch, two GEMMs, combine; with the
+    automatic token-tile choice on bf16 weights each GEMM launches both forms
+    (the one not chosen returns at once)."""
+    both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
+    return 5 + (2 if both else 0)
 
 
 # ---------------------------------------------------------------- main --
@@ -306,8 +322,8 @@ def main():
 
     t_max = max_over_ranks(sum(step_ms), dist, dev)
     flops = wl.flops
-    value = world * K * flops / (t_max / 1e3) / 1e12
-    tok_s = world * K * T / (t_max / 1e3)
+    value = job_throughput(world, K, flops, t_max) / 1e12
+    tok_s = job_throughput(world, K, T, t_max)
     wbytes = touched * 3 * d * f * (1 if wl.dtype == "bf16_int8w" else 2)
     roofline = roofline_entry(wl, pk, stage_ms, touched, clocks)
 
@@ -339,8 +355,9 @@ def main():
         "hbm_gbs_weights": round(world * K * wbytes / (t_max / 1e3) / 1e9, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,
-        "gpu_launches": 5 * K,
-        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
+        "gpu_launches": launches_per_step(wl, a.path) * K,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                   "power_w_max": clocks.get("power_w_max"), "samples": clocks.get("samples")},
         "wall_s_timed_region": round(wall, 3),
     }
     if e2e:

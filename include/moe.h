@@ -196,6 +196,18 @@ MOE_EXPORT moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_op
  * code != NULL) or MOE_ERR_CUDA. */
 MOE_EXPORT moe_status_t moe_device_status(const void* workspace, moe_stream_t stream, uint32_t* code);
 
+/* Check of the failure path, with no fault: launches one thread that waits,
+ * with the same bounded mbarrier wait the GEMM pipelines use, on a barrier that
+ * nothing arrives on, giving up after `limit_us` microseconds (1 .. 10^7). The
+ * kernel then records bit 0x10 in the status word at the start of `workspace`
+ * (device memory, 256-byte aligned, at least 256 bytes) and returns, so a
+ * following moe_device_status(workspace, stream, &code) returns
+ * MOE_ERR_DEVICE_CHECK with code 0x10 and the context stays usable. No
+ * counterpart on the pages: it exercises the library's own time limits.
+ * Returns MOE_OK once launched, MOE_ERR_WORKSPACE / MOE_ERR_INVALID_ARG on bad
+ * arguments, MOE_ERR_CUDA if the launch fails. */
+MOE_EXPORT moe_status_t moe_selftest_bounded_wait(void* workspace, uint32_t limit_us, moe_stream_t stream);
+
 /* Static description of a status code (never NULL). */
 MOE_EXPORT const char* moe_status_string(moe_status_t status);
 

@@ -19,7 +19,8 @@ from ._native import (  # noqa: F401
 )
 
 __all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_forward_noalloc", "moe_workspace_size",
-           "moe_device_status", "moe_status_string", "moe_abi_version", "dtype_code"]
+           "moe_device_status", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
+           "dtype_code"]
 
 
 class MoeError(RuntimeError):
@@ -159,6 +160,14 @@ def moe_forward_noalloc(x, w_router, w_gate, w_up, w_down, out, scales=None, rou
     if st != N.MOE_OK and raise_on_error:
         raise MoeError(st, "moe_forward_noalloc")
     return st
+
+
+def moe_selftest_bounded_wait(workspace, limit_us=1000, stream=None):
+    """Launch the failure-path check: a bounded wait that nothing satisfies,
+    recording status bit 0x10 in ``workspace`` (read it with moe_device_status)."""
+    st = N.lib().moe_selftest_bounded_wait(_ptr(workspace), limit_us, _stream(stream))
+    if st != N.MOE_OK:
+        raise MoeError(st, "moe_selftest_bounded_wait")
 
 
 def moe_device_status(workspace=None, stream=None):

@@ -53,6 +53,7 @@ EXPORTS.update({
                                c_void_p]),
     "moe_forward_noalloc": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), c_void_p]),
     "moe_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_uint32)]),
+    "moe_selftest_bounded_wait": (c_int, [c_void_p, c_uint32, c_void_p]),
     "moe_status_string": (c_char_p, [c_int]),
     "moe_abi_version": (c_int32, []),
 })

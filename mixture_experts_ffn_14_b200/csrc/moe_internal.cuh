@@ -23,6 +23,7 @@ enum : uint32_t {
   kStatusMmaTimeout = 1u << 1,
   kStatusEpilogueTimeout = 1u << 2,
   kStatusConvertTimeout = 1u << 3,
+  kStatusSelftestTimeout = 1u << 4,
 };
 
 // Byte offsets of the regions of one call's workspace (each 256-aligned).

@@ -138,3 +138,11 @@ def test_option_checks():
     assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED
     bad = N.MoeOptions(0, None, 0, 0, None, 0, 0x50000008, None, 0.0)
     assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED
+
+
+def test_selftest_argument_checks():
+    f = N.lib().moe_selftest_bounded_wait
+    assert f(None, 1000, None) == N.MOE_ERR_WORKSPACE
+    assert f(0x20000010, 1000, None) == N.MOE_ERR_WORKSPACE      # not 256-byte aligned
+    assert f(0x20000000, 0, None) == N.MOE_ERR_INVALID_ARG
+    assert f(0x20000000, 20_000_000, None) == N.MOE_ERR_INVALID_ARG
