@@ -118,7 +118,7 @@ def test_bf16_erf_gelu():
 
 # ------------------------------------------------------------------ int8 --
 
-@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("path", PATHS + [moe.MOE_PATH_AUTO])
 @pytest.mark.parametrize("T", [5, 300])
 def test_int8_parity_all_paths(T, path):
     inp = small_bf16(T, seed=21, int8=True)
@@ -228,3 +228,22 @@ def test_renormalized_gates_sum_to_one():
     inp = small_bf16(64, seed=70)
     gpu = run_gpu(inp, renormalize=True, want_h=False)
     assert np.abs(gpu["gates"].sum(1) - 1.0).max() < 1e-6
+
+
+@pytest.mark.parametrize("T", [1, 129, 256, 257, 300, 384, 385])
+def test_int8_tile_boundaries(T):
+    # Every token picks experts 0 and 1 (T rows each): full and ragged 128-row
+    # tiles on the automatic path (weight-stream at T <= 256, token tiles above)
+    # and on forced single-CTA token tiles.
+    inp = small_bf16(T, seed=90, int8=True)
+    inp["router_bias"] = torch.tensor([40.0, 30.0, 0, 0, 0, 0, 0, 0], device=DEV)
+    for path in (moe.MOE_PATH_AUTO, moe.MOE_PATH_TOKEN_TILE_SINGLE):
+        gpu = run_gpu(inp, path=path)
+        assert list(gpu["counts"][:2]) == [T, T]
+        full_check(inp, gpu)
+
+
+@pytest.mark.parametrize("splits", [2, 3])
+def test_int8_token_tile_split_k(splits):
+    inp = small_bf16(600, d=512, f=384, seed=91, int8=True)
+    full_check(inp, run_gpu(inp, down_splits=splits))
