@@ -345,15 +345,8 @@ template <int KIND, bool WS, bool W8>
 cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   using C = Cfg<W8>;
   auto kern = moe_expert_gemm_kernel<KIND, WS, W8>;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  const cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (err != cudaSuccess) return err;
-    configured_device = dev;
-  }
 
   CUtensorMap tm_x, tm_w0, tm_w1;
   {

@@ -299,10 +299,7 @@ template <int KIND, bool W8>
 cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   using C = PairCfg<W8>;
   auto kern = moe_expert_gemm_pair_kernel<KIND, W8>;
-  static int configured_device = -1;
-  static int max_pairs = 0;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  const cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
 
   cudaLaunchAttribute attr[1];
@@ -317,15 +314,24 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
 
-  if (configured_device != dev) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (err != cudaSuccess) return err;
-    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+  // Clusters of two that fit at once on this device (queried once per device).
+  const int max_pairs = once_per_device(reinterpret_cast<const void*>(&launch_pair<KIND, W8>), [](const void*) {
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 2;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+    c.blockDim = dim3(PairCfg<W8>::THREADS, 1, 1);
+    c.dynamicSmemBytes = PairCfg<W8>::SMEM;
+    c.attrs = &at;
+    c.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = device_sm_count() / 2;
-    max_pairs = n;
-    configured_device = dev;
-  }
+    if (cudaOccupancyMaxActiveClusters(&n, moe_expert_gemm_pair_kernel<KIND, W8>, &c) != cudaSuccess || n <= 0)
+      n = device_sm_count() / 2;
+    return n;
+  });
 
   CUtensorMap tm_x, tm_w0, tm_w1;
   {

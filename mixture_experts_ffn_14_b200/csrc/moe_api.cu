@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <vector>
 
@@ -92,6 +93,40 @@ int device_sm_count() {
     g_sm_count[dev] = n;
   }
   return g_sm_count[dev];
+}
+
+int once_per_device(const void* key, int (*setup)(const void* key)) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto k = std::make_pair(key, dev);
+  const auto it = cache.find(k);
+  if (it != cache.end()) return it->second;
+  const int v = setup(key);
+  if (v >= 0) cache[k] = v;
+  return v;
+}
+
+cudaError_t set_smem_limit_once(const void* kern, int bytes) {
+  // The kernels' limits are fixed per kernel, so the byte count is looked up
+  // through a small registry keyed by the kernel.
+  static std::mutex mu;
+  static std::map<const void*, int> wanted;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    wanted[kern] = bytes;
+  }
+  const int r = once_per_device(kern, [](const void* k) -> int {
+    int b = 0;
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      b = wanted[k];
+    }
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess ? 1 : -1;
+  });
+  return r > 0 ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const void* base,

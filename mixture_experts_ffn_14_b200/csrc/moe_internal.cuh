@@ -105,4 +105,12 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, 
 
 int device_sm_count();
 
+// Host: run `setup` once per (key, current device) and cache its value; the
+// first call on a device pays, later calls (from any thread) read the cache.
+// A negative result is an error and is not cached.
+int once_per_device(const void* key, int (*setup)(const void* key));
+
+// Host: raise a kernel's dynamic shared-memory limit once per device.
+cudaError_t set_smem_limit_once(const void* kern, int bytes);
+
 }  // namespace moe
