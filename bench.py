@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--f", type=int, default=None, help="override the expert width")
     ap.add_argument("--path", choices=["auto", "token_tile", "weight_stream", "token_tile_single"], default="auto",
                     help="kernel family (default: the library's automatic choice)")
+    ap.add_argument("--row-gather", action="store_true",
+                    help="token tiles gather their gate/up rows from x (TMA row gather) instead of the copy")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode (T=64) side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
@@ -67,7 +69,10 @@ def peaks():
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """nvidia-smi samples every 100 ms; only those taken inside the `with` block count.
+
+    Entering waits (up to 10 s) until nvidia-smi has produced its first sample, so
+    that sampling is live when the timed region starts."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -78,31 +83,53 @@ class ClockSampler:
 
         self.proc = None
         self.lines = []
+        self._stamped = []
+        self._reader = None
+        self._t0 = self._t1 = None
         try:
             pr = torch.cuda.get_device_properties(torch_dev)
             self.bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
         except Exception:
             self.bus = None
 
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self._stamped.append((time.perf_counter(), ln))
+
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        import threading
+
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.bus:
             cmd += ["-i", self.bus]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._reader = threading.Thread(target=self._read, daemon=True)
+            self._reader.start()
+            deadline = time.perf_counter() + 10.0
+            while not self._stamped and time.perf_counter() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+        self._t0 = time.perf_counter()
         return self
 
     def __exit__(self, *exc):
+        self._t1 = time.perf_counter()
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self._reader is not None:
+                self._reader.join(timeout=5)
+        inside = [ln for t, ln in self._stamped if self._t0 <= t <= self._t1 + 0.05]
+        # Keep at least the newest sample taken before the region if none fell inside.
+        if not inside and self._stamped:
+            inside = [self._stamped[-1][1]]
+        self.lines = inside
 
     def summary(self):
         sm, smax, power, reasons = [], None, [], set()
@@ -190,10 +217,11 @@ class Runner:
 
     PATHS = {"auto": 0, "token_tile": 1, "weight_stream": 2, "token_tile_single": 3}
 
-    def __init__(self, moe, inp, T, d, f, dev, path="auto"):
+    def __init__(self, moe, inp, T, d, f, dev, path="auto", row_gather=False):
         import torch
 
         self.moe, self.inp = moe, inp
+        self.row_gather = row_gather
         self.path = self.PATHS[path]
         dt = moe.dtype_code(inp["x"], inp["w_gate"])
         self.ws = torch.empty(moe.moe_workspace_size(T, d, f, dtype=dt, path=self.path), dtype=torch.uint8,
@@ -204,7 +232,7 @@ class Runner:
         i = self.inp
         self.moe.moe_forward_ex(x, i["w_router"], i["w_gate"], i["w_up"], i["w_down"], out, self.ws,
                                 scales=self.scales, router_bias=i.get("router_bias"), stage_events=events,
-                                debug=debug, path=self.path)
+                                debug=debug, path=self.path, row_gather=self.row_gather)
 
 
 def timed_steps(run, x, out, K, flush, clk=None):
@@ -292,7 +320,7 @@ def main():
 
     T, d, f = wl.T, wl.d, wl.f
     inp = W.make_torch(wl, dev)
-    run = Runner(moe, inp, T, d, f, dev, a.path)
+    run = Runner(moe, inp, T, d, f, dev, a.path, a.row_gather)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     counts = torch.empty(8, dtype=torch.int32, device=dev)
@@ -352,6 +380,7 @@ def main():
         "tokens_per_s": round(tok_s, 1),
         "expert_slots": expert_counts,
         "path": a.path,
+        "row_gather": bool(a.row_gather),
         "hbm_gbs_weights": round(world * K * wbytes / (t_max / 1e3) / 1e9, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,

@@ -85,10 +85,11 @@ typedef enum {
 } moe_activation_t;
 
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
- * down projection) when the average tokens per expert is small, else
- * TOKEN_TILE (256-token tiles on the MMA M side of a CTA pair, cta_group::2).
- * TOKEN_TILE_SINGLE runs 128-token tiles on single CTAs (kept for comparison).
- * All compute the same result. */
+ * down projection) when the average tokens per expert is small (T <= 256),
+ * else token tiles (tokens on the MMA M side), where the device chooses from
+ * the expert counts between 128-token tiles on single CTAs and 256-token tiles
+ * on CTA pairs (cta_group::2). TOKEN_TILE forces the pair form,
+ * TOKEN_TILE_SINGLE the single-CTA form. All compute the same result. */
 typedef enum {
   MOE_PATH_AUTO = 0,
   MOE_PATH_TOKEN_TILE = 1,
@@ -136,6 +137,11 @@ typedef struct {
   const float* post_norm_weight; /* [d] fp32 RMSNorm weight applied to the sublayer
                                   output before the residual add, or NULL (no norm)      */
   float norm_eps;              /* RMSNorm epsilon (> 0) when post_norm_weight is set      */
+  int32_t row_gather;          /* 0: token tiles read a permuted copy of x made by the
+                                  dispatch stage (default); 1: they gather their gate/up
+                                  operand rows from x with TMA row gathers (no copy; slower
+                                  on B200, where four-row gathers cannot feed the MMA).
+                                  The weight-stream form always reads the copy.           */
 } moe_options_t;
 
 /* Optional outputs for inspection; each is a device pointer or NULL.

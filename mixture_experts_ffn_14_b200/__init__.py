@@ -94,7 +94,7 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, out, scales=None, stream=None
 
 
 def _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual, post_norm_weight,
-             norm_eps):
+             norm_eps, row_gather=False):
     ev = None
     if stage_events is not None:
         handles = [e.cuda_event for e in stage_events]
@@ -103,20 +103,23 @@ def _options(activation, router_bias, path, down_splits, stage_events, renormali
         ev = (ctypes.c_void_p * 6)(*handles)
     opts = N.MoeOptions(activation, _ptr(router_bias), path, down_splits,
                         ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)) if ev is not None else None,
-                        int(bool(renormalize)), _ptr(residual), _ptr(post_norm_weight), float(norm_eps))
+                        int(bool(renormalize)), _ptr(residual), _ptr(post_norm_weight), float(norm_eps),
+                        int(bool(row_gather)))
     return opts, ev
 
 
 def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=None, router_bias=None,
                    activation=MOE_ACT_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, debug=None, stream=None,
                    stage_events=None, renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5,
-                   raise_on_error=True):
+                   row_gather=False, raise_on_error=True):
     """Forward pass on a caller workspace (a uint8 CUDA tensor). ``debug`` is a
     dict with any of idx, gates, counts, offsets, perm_token, perm_slot, h.
     ``stage_events``: 6 torch.cuda.Event (already created, e.g. recorded once)
     that the library records around its five stages. ``renormalize``,
     ``activation``, ``residual``, ``post_norm_weight`` / ``norm_eps``: the
-    moe_options_t variants (Mixtral routing, SiLU, post-RMSNorm + residual)."""
+    moe_options_t variants (Mixtral routing, SiLU, post-RMSNorm + residual).
+    ``row_gather``: token tiles gather their gate/up rows from x with TMA row
+    gathers instead of reading the dispatch stage's permuted copy."""
     T, d = x.shape
     E, _, f = w_gate.shape
     sc = _scales(scales)
@@ -124,7 +127,7 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
                      ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
                      dtype_code(x, w_gate))
     opts, _keep = _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual,
-                           post_norm_weight, norm_eps)
+                           post_norm_weight, norm_eps, row_gather)
     dbg = None
     if debug:
         dbg = N.MoeDebug(*[_ptr(debug.get(n)) for n in

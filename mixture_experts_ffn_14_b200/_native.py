@@ -37,7 +37,7 @@ class MoeArgs(ctypes.Structure):
 class MoeOptions(ctypes.Structure):
     _fields_ = [("activation", c_int), ("router_bias", c_void_p), ("path", c_int), ("down_splits", c_int32),
                 ("stage_events", POINTER(c_void_p)), ("renormalize", c_int32), ("residual", c_void_p),
-                ("post_norm_weight", c_void_p), ("norm_eps", c_float)]
+                ("post_norm_weight", c_void_p), ("norm_eps", c_float), ("row_gather", c_int32)]
 
 
 class MoeDebug(ctypes.Structure):

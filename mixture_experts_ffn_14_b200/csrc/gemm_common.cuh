@@ -30,6 +30,7 @@ struct Params {
   const int32_t* counts;
   const int32_t* offsets;
   const float* gate_perm;
+  const int32_t* row_token;  // GATEUP token tiles: token of each permuted row, A rows gathered from x
   const __nv_bfloat16* s0;
   const __nv_bfloat16* s1;
   void* out;
@@ -83,6 +84,17 @@ struct SharedSched {
 struct Tile {
   int e, row0, rows, n0, kb0;
 };
+
+// Token ids of one producer lane's four A rows (permuted rows q0 .. q0+3 of a
+// tile whose valid rows are [t.row0, t.row0 + t.rows)). Rows past the expert's
+// count repeat the tile's first token: they are computed and never stored.
+__device__ __forceinline__ void gather_rows(const Params& p, const Tile& t, int q0, int32_t r[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int q = q0 + j;
+    r[j] = __ldg(p.row_token + (q < t.row0 + t.rows ? q : t.row0));
+  }
+}
 
 // Row tiles of `tile_rows` per expert, column tiles of p.ntile, splits; row
 // tile fastest so that concurrently running CTAs share weight tiles in L2.

@@ -107,36 +107,46 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0) {
-      // Weight-stream tiles read each weight byte once: mark it evict-first so
-      // it does not push the reused activations out of L2.
-      const uint64_t wpolicy = policy_evict_first();
-      auto load_w = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int n, int k, int e) {
-        if (WS) tma_load_3d_hint(dst, map, bar, n, k, e, wpolicy);
-        else tma_load_3d(dst, map, bar, n, k, e);
-      };
-      int stage = 0;
-      uint32_t phase = 0;
-      Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
-        const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
-        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
-        const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
-        for (int kb = 0; kb < p.kb_per_split; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) || *abort_flag) {
+    // Lane 0 waits for a free stage, arms its full barrier and loads the weight
+    // boxes (and the activation box of materialised rows). With the row gather
+    // each of the 32 lanes also loads four token rows of A straight from x.
+    const bool gather = !WS && KIND == GATEUP && p.row_token != nullptr;
+    // Weight-stream tiles read each weight byte once: mark it evict-first so
+    // it does not push the reused activations out of L2.
+    const uint64_t wpolicy = policy_evict_first();
+    auto load_w = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int n, int k, int e) {
+      if (WS) tma_load_3d_hint(dst, map, bar, n, k, e, wpolicy);
+      else tma_load_3d(dst, map, bar, n, k, e);
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    Tile t;
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+      int32_t rtok[4] = {0, 0, 0, 0};
+      if (gather) gather_rows(p, t, t.row0 + 4 * lane, rtok);
+      const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
+      const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
+      const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
+      for (int kb = 0; kb < p.kb_per_split; ++kb) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (lane == 0) {
             atomicOr(p.status, kStatusProducerTimeout);
             *abort_flag = 1;
-            goto producer_done;
           }
-          uint8_t* xs = smem + stage * C::STAGE_BYTES;
-          uint8_t* ws = xs + X_BYTES;
-          uint8_t* w8 = ws + W_BYTES;
-          const int k0 = (t.kb0 + kb) * BK;
+          goto producer_done;
+        }
+        uint8_t* xs = smem + stage * C::STAGE_BYTES;
+        uint8_t* ws = xs + X_BYTES;
+        uint8_t* w8 = ws + W_BYTES;
+        const int k0 = (t.kb0 + kb) * BK;
+        if (lane == 0) {
           mbar_arrive_expect_tx(&full_bar[stage], xbytes + wbytes);
           if (WS) {
             for (int b = 0; b < nbox_x; ++b)
               tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
-          } else {
+          } else if (!gather) {
             tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
           }
           if (W8) {
@@ -159,14 +169,17 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
                 load_w(ws + j * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64 * j, k0, t.e);
             }
           }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+        }
+        __syncwarp();  // the barrier is armed before any lane's gather can complete on it
+        // Lane l fills A rows 4l .. 4l+3 (512 B, 128-B swizzled like one tall box).
+        if (gather) tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-    producer_done:;
     }
+  producer_done:;
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
@@ -350,9 +363,11 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
 
   CUtensorMap tm_x, tm_w0, tm_w1;
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.rows)};
+    // Row gather: the map covers x itself and its box is one row high.
+    const bool gather = !WS && KIND == GATEUP && a.row_token != nullptr;
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(gather ? a.x_rows : a.rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
-    const uint32_t box[2] = {BK, static_cast<uint32_t>(WS ? XBOX_ROWS_WS : BM)};
+    const uint32_t box[2] = {BK, static_cast<uint32_t>(gather ? 1 : WS ? XBOX_ROWS_WS : BM)};
     if (!encode_tensor_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -373,6 +388,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.counts = a.counts;
   p.offsets = a.offsets;
   p.gate_perm = a.gate_perm;
+  p.row_token = (!WS && KIND == GATEUP) ? a.row_token : nullptr;
   p.s0 = a.s0;
   p.s1 = a.s1;
   p.out = a.out;

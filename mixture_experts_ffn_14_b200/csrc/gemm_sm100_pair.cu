@@ -125,47 +125,65 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      Tile t;
-      for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
-        const int row = t.row0 + BM * static_cast<int>(rank);
-        // GATEUP: the even CTA holds the gate columns, the odd one the up
-        // columns (accumulator columns 0..127 / 128..255). DOWN: 128 columns each.
-        const CUtensorMap* wmap = (KIND == GATEUP && rank == 1) ? &tm_w1 : &tm_w0;
-        const int n = KIND == GATEUP ? t.n0 : t.n0 + 128 * static_cast<int>(rank);
-        for (int kb = 0; kb < p.kb_per_split; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) || *abort_flag) {
+    // Lane 0 waits for a free stage, arms the barrier and loads the weight box
+    // (and the activation box of materialised rows); with the row gather each
+    // of the 32 lanes also loads four of this CTA's 128 token rows from x.
+    const bool gather = KIND == GATEUP && p.row_token != nullptr;
+    int stage = 0;
+    uint32_t phase = 0;
+    Tile t;
+    for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
+      const int row = t.row0 + BM * static_cast<int>(rank);
+      int32_t rtok[4] = {0, 0, 0, 0};
+      if (gather) gather_rows(p, t, row + 4 * lane, rtok);
+      // GATEUP: the even CTA holds the gate columns, the odd one the up
+      // columns (accumulator columns 0..127 / 128..255). DOWN: 128 columns each.
+      const CUtensorMap* wmap = (KIND == GATEUP && rank == 1) ? &tm_w1 : &tm_w0;
+      const int n = KIND == GATEUP ? t.n0 : t.n0 + 128 * static_cast<int>(rank);
+      for (int kb = 0; kb < p.kb_per_split; ++kb) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (lane == 0) {
             atomicOr(p.status, kStatusProducerTimeout);
             *abort_flag = 1;
-            goto producer_done;
           }
-          {
-            uint8_t* xs = smem + stage * C::STAGE_BYTES;
-            uint8_t* ws = xs + X_BYTES;
-            uint8_t* w8 = ws + PW_BYTES;
-            const int k0 = (t.kb0 + kb) * BK;
-            if (W8) {
+          goto producer_done;
+        }
+        {
+          uint8_t* xs = smem + stage * C::STAGE_BYTES;
+          uint8_t* ws = xs + X_BYTES;
+          uint8_t* w8 = ws + PW_BYTES;
+          const int k0 = (t.kb0 + kb) * BK;
+          if (W8) {
+            if (lane == 0) {
               mbar_arrive_expect_tx(&full_bar[stage], X_BYTES + PW8_BYTES);
-              tma_load_2d(xs, &tm_x, &full_bar[stage], k0, row);
+              if (!gather) tma_load_2d(xs, &tm_x, &full_bar[stage], k0, row);
               tma_load_3d(w8, wmap, &full_bar[stage], n, k0, t.e);
-            } else {
-              const uint32_t bar0 = mapa_shared(&full_bar[stage], 0);
+            }
+            __syncwarp();  // armed before any lane's gather can complete on it
+            if (gather) tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+          } else {
+            const uint32_t bar0 = mapa_shared(&full_bar[stage], 0);
+            if (lane == 0) {
               if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (X_BYTES + PW_BYTES));
-              tma_load_2d_pair(xs, &tm_x, bar0, k0, row);
+              if (!gather) tma_load_2d_pair(xs, &tm_x, bar0, k0, row);
               tma_load_3d_pair(ws, wmap, bar0, n, k0, t.e);
               tma_load_3d_pair(ws + WCHUNK, wmap, bar0, n + 64, k0, t.e);
             }
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
+            __syncwarp();
+            if (gather) tma_gather4_pair(xs + lane * 512, &tm_x, bar0, k0, rtok[0], rtok[1], rtok[2], rtok[3]);
           }
         }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
-      // Drain: every stage's last release (an arrive sent by the pair's MMA
-      // commit) has landed before this CTA may exit.
+    }
+    // Drain: every stage's last release (an arrive sent by the pair's MMA
+    // commit) has landed before this CTA may exit.
+    if (lane == 0) {
       for (int i = 0; i < STAGES; ++i) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs)) {
           atomicOr(p.status, kStatusProducerTimeout);
@@ -176,8 +194,8 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
           phase ^= 1;
         }
       }
-    producer_done:;
     }
+  producer_done:;
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0 && rank == 0) {
@@ -335,9 +353,11 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
 
   CUtensorMap tm_x, tm_w0, tm_w1;
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.rows)};
+    // Row gather: the map covers x itself and its box is one row high.
+    const bool gather = KIND == GATEUP && a.row_token != nullptr;
+    const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(gather ? a.x_rows : a.rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
-    const uint32_t box[2] = {BK, BM};
+    const uint32_t box[2] = {BK, static_cast<uint32_t>(gather ? 1 : BM)};
     if (!encode_tensor_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -358,6 +378,7 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   p.counts = a.counts;
   p.offsets = a.offsets;
   p.gate_perm = a.gate_perm;
+  p.row_token = KIND == GATEUP ? a.row_token : nullptr;
   p.s0 = a.s0;
   p.s1 = a.s1;
   p.out = a.out;

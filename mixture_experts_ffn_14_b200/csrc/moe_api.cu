@@ -219,6 +219,7 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   const int64_t rows = 2 * T;
   L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
   L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path);
+  L.tile_path = dtype != MOE_F32 && !L.weight_stream;
   if (dtype == MOE_F32) {
     L.splits = 1;
   } else if (L.weight_stream) {
@@ -274,6 +275,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     return MOE_ERR_MISALIGNED;
   if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE) return MOE_ERR_INVALID_ARG;
   if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
+  if (o->row_gather != 0 && o->row_gather != 1) return MOE_ERR_INVALID_ARG;
   if (o->router_bias && !aligned16(o->router_bias)) return MOE_ERR_MISALIGNED;
   const bool h_ext = dbg && dbg->h;
   if (h_ext && !aligned16(dbg->h)) return MOE_ERR_MISALIGNED;
@@ -295,7 +297,10 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   int32_t* perm_slot = reinterpret_cast<int32_t*>(ws + L.perm_slot);
   int32_t* slot_pos = reinterpret_cast<int32_t*>(ws + L.slot_pos);
   float* gate_perm = reinterpret_cast<float*>(ws + L.gate_perm);
-  void* xp = ws + L.xp;
+  // With the row gather the token-tile GEMM reads x itself and the dispatch
+  // stage skips the permuted copy.
+  const bool gather_x = L.tile_path && o->row_gather == 1;
+  void* xp = gather_x ? nullptr : static_cast<void*>(ws + L.xp);
   void* h = h_ext ? dbg->h : static_cast<void*>(ws + L.h);
   float* y = reinterpret_cast<float*>(ws + L.y);
   const int64_t T = a->T, d = a->d, f = a->f;
@@ -327,7 +332,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   } else {
     const bool w8 = a->dtype == MOE_BF16_INT8W;
     TcGemmArgs g{};
-    g.x = xp;
+    g.x = gather_x ? a->x : xp;
+    g.row_token = gather_x ? perm_token : nullptr;
+    g.x_rows = T;
     g.w0 = a->w_gate;
     g.w1 = a->w_up;
     g.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_gate) : nullptr;
@@ -369,6 +376,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     MOE_TRY(mark(3));
     TcGemmArgs g2 = g;
     g2.x = h;
+    g2.row_token = nullptr;
     g2.w0 = a->w_down;
     g2.w1 = nullptr;
     g2.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_down) : nullptr;

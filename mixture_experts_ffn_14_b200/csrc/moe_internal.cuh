@@ -35,6 +35,7 @@ struct WorkspaceLayout {
   int32_t splits;    // split-K factor of the down projection
   int32_t router_slices;  // d slices of the router grid
   bool weight_stream;
+  bool tile_path;    // token tiles (bf16 / int8 weights, not weight-stream): row gather possible
 };
 
 // Host: workspace layout for a call (valid arguments assumed).
@@ -58,7 +59,7 @@ cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_route
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
-                            float* gate_perm, void* xp, cudaStream_t s);
+                            float* gate_perm, void* xp, cudaStream_t s);  // xp == nullptr: no row copy
 
 // out[t] = residual[t] + norm(y0 + y1); residual and norm_weight may be NULL.
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
@@ -74,7 +75,9 @@ cudaError_t launch_f32_down(const float* h, const float* wd, const int32_t* coun
 
 // tcgen05 grouped expert GEMMs (bf16 or int8 weights).
 struct TcGemmArgs {
-  const void* x;            // [rows, K] bf16 activations (Xp or H), rows = 2T
+  const void* x;            // [rows, K] bf16 activations (Xp or H), rows = 2T; x [x_rows, K] with row_token
+  const int32_t* row_token; // GATEUP token tiles: token of each permuted row (A rows gathered from x), or nullptr
+  int64_t x_rows;           // rows of x when row_token is set (T)
   const void* w0;           // [E, K, N] gate (GATEUP) or down (DOWN) weights, bf16 or int8
   const void* w1;           // [E, K, N] up weights (GATEUP) or nullptr
   const __nv_bfloat16* s0;  // int8: [E, N] scales of w0, else nullptr

@@ -311,6 +311,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     pos_sm[lane][1] = pb;
   }
   __syncthreads();
+  if (xp == nullptr) return;  // the expert GEMM gathers the rows itself
 
   // Gather: 64 rows of d elements, as 16-byte vectors; eight loads in flight
   // per thread before their stores.
@@ -503,7 +504,9 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
                             float* gate_perm, void* xp, cudaStream_t s) {
-  const int64_t g = std::min<int64_t>(16, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk));
+  // Extra CTAs along y only split the row gather; without Xp one suffices.
+  const int64_t g =
+      xp ? std::min<int64_t>(16, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk)) : 1;
   const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(g), 1);
   if (dtype == MOE_F32)
     moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(

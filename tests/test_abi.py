@@ -138,6 +138,8 @@ def test_option_checks():
     assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED
     bad = N.MoeOptions(0, None, 0, 0, None, 0, 0x50000008, None, 0.0)
     assert _call(a, opts=bad) == N.MOE_ERR_MISALIGNED
+    bad = N.MoeOptions(0, None, 0, 0, None, 0, None, None, 0.0, 2)   # row_gather must be 0 or 1
+    assert _call(a, opts=bad) == N.MOE_ERR_INVALID_ARG
 
 
 def test_selftest_argument_checks():

@@ -60,6 +60,53 @@ def test_bf16_parity_all_paths(T, path):
     full_check(inp, run_gpu(inp, path=path))
 
 
+# Row gather (moe_options_t.row_gather): token tiles read the gate/up operand
+# rows from x with TMA four-row gathers instead of the dispatch stage's copy.
+TT_PATHS = [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE, moe.MOE_PATH_AUTO]
+
+
+@pytest.mark.parametrize("path", TT_PATHS)
+@pytest.mark.parametrize("T", [1, 37, 129, 257, 1000])
+def test_row_gather_parity(T, path):
+    inp = small_bf16(T, seed=31)
+    full_check(inp, run_gpu(inp, path=path, row_gather=True))
+
+
+@pytest.mark.parametrize("path", TT_PATHS)
+def test_row_gather_from_an_offset_view_of_x(path):
+    # x is a 16-byte aligned view three rows into a larger buffer whose other
+    # rows hold 1000.0: reading any row outside the view would show in the output.
+    inp = small_bf16(300, seed=21)
+    T, d = inp["x"].shape
+    big = torch.full((T + 7, d), 1000.0, dtype=inp["x"].dtype, device=DEV)
+    big[3:3 + T] = inp["x"]
+    view = big[3:3 + T]
+    assert view.is_contiguous() and view.data_ptr() % 16 == 0
+    inp2 = dict(inp, x=view)
+    full_check(inp2, run_gpu(inp2, path=path, row_gather=True))
+
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE])
+@pytest.mark.parametrize("T", [5, 300])
+def test_row_gather_int8(T, path):
+    inp = small_bf16(T, seed=33, int8=True)
+    full_check(inp, run_gpu(inp, path=path, row_gather=True))
+
+
+def test_row_gather_matches_copy_bitwise():
+    # Same rows, same MMA order: the two ways of feeding A give identical bits.
+    inp = small_bf16(700, seed=35)
+    a = run_gpu(inp, path=moe.MOE_PATH_AUTO)
+    b = run_gpu(inp, path=moe.MOE_PATH_AUTO, row_gather=True)
+    assert np.array_equal(a["out"], b["out"])
+    assert torch.equal(a["h"], b["h"])
+
+
+def test_row_gather_skewed_with_empty_experts():
+    inp = small_bf16(400, seed=37, skew=True)
+    full_check(inp, run_gpu(inp, row_gather=True))
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3])
 def test_bf16_weight_stream_split_k(splits):
     inp = small_bf16(90, d=256, f=384)

@@ -71,7 +71,7 @@ def test_noalloc_f32_and_token_tile_path():
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
-    w = W.Workload("noalloc_big", 4096, 512, 1024, dtype="bf16", seed=43)
+    w = W.Workload("noalloc_big", 4096, 512, 2048, dtype="bf16", seed=43)
     inp = W.make_torch(w, DEV)
     out = torch.empty_like(inp["x"])
     st = moe.moe_forward_noalloc(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out,
