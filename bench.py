@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import dataclasses
+import datetime
 import json
 import os
 import statistics
@@ -69,12 +70,11 @@ def peaks():
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi samples every 100 ms; only those taken inside the `with` block count.
+    """nvidia-smi samples every 100 ms; only those whose own timestamp falls
+    inside the `with` block count (its output reaches the pipe in blocks, so the
+    arrival time of a line says nothing)."""
 
-    Entering waits (up to 10 s) until nvidia-smi has produced its first sample, so
-    that sampling is live when the timed region starts."""
-
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -83,8 +83,6 @@ class ClockSampler:
 
         self.proc = None
         self.lines = []
-        self._stamped = []
-        self._reader = None
         self._t0 = self._t1 = None
         try:
             pr = torch.cuda.get_device_properties(torch_dev)
@@ -92,43 +90,41 @@ class ClockSampler:
         except Exception:
             self.bus = None
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            if ln.strip():
-                self._stamped.append((time.perf_counter(), ln))
-
     def __enter__(self):
-        import threading
-
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.bus:
             cmd += ["-i", self.bus]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._reader = threading.Thread(target=self._read, daemon=True)
-            self._reader.start()
-            deadline = time.perf_counter() + 10.0
-            while not self._stamped and time.perf_counter() < deadline and self.proc.poll() is None:
-                time.sleep(0.01)
+            time.sleep(0.5)  # let it start sampling before the region opens
         except Exception:
             self.proc = None
-        self._t0 = time.perf_counter()
+        self._t0 = time.time()
         return self
 
     def __exit__(self, *exc):
-        self._t1 = time.perf_counter()
-        if self.proc is not None:
-            self.proc.terminate()
+        self._t1 = time.time()
+        if self.proc is None:
+            return
+        time.sleep(0.15)  # one more sample period
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        stamped = []
+        for ln in out.splitlines():
+            ts = ln.split(",", 1)[0].strip()
             try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            if self._reader is not None:
-                self._reader.join(timeout=5)
-        inside = [ln for t, ln in self._stamped if self._t0 <= t <= self._t1 + 0.05]
-        # Keep at least the newest sample taken before the region if none fell inside.
-        if not inside and self._stamped:
-            inside = [self._stamped[-1][1]]
+                t = datetime.datetime.strptime(ts, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            stamped.append((t, ln.split(",", 1)[1]))
+        inside = [ln for t, ln in stamped if self._t0 <= t <= self._t1]
+        if not inside and stamped:  # region shorter than a sample period: the nearest sample
+            mid = 0.5 * (self._t0 + self._t1)
+            inside = [min(stamped, key=lambda tl: abs(tl[0] - mid))[1]]
         self.lines = inside
 
     def summary(self):
@@ -339,10 +335,10 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    wall0 = time.perf_counter()
     with ClockSampler(dev) as clk:
+        wall0 = time.perf_counter()
         step_ms, stage_ms = timed_steps(run, inp["x"], out, K, flush)
-    wall = time.perf_counter() - wall0
+        wall = time.perf_counter() - wall0
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()

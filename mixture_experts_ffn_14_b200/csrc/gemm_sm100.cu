@@ -33,6 +33,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "gemm_common.cuh"
 
@@ -110,7 +111,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     // Lane 0 waits for a free stage, arms its full barrier and loads the weight
     // boxes (and the activation box of materialised rows). With the row gather
     // each of the 32 lanes also loads four token rows of A straight from x.
-    const bool gather = !WS && KIND == GATEUP && p.row_token != nullptr;
+    // The two variants are compiled separately: the plain one is lane 0 alone
+    // with no warp-synchronous step, so its refill latency stays minimal.
     // Weight-stream tiles read each weight byte once: mark it evict-first so
     // it does not push the reused activations out of L2.
     const uint64_t wpolicy = policy_evict_first();
@@ -118,68 +120,78 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       if (WS) tma_load_3d_hint(dst, map, bar, n, k, e, wpolicy);
       else tma_load_3d(dst, map, bar, n, k, e);
     };
-    int stage = 0;
-    uint32_t phase = 0;
-    Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
-      int32_t rtok[4] = {0, 0, 0, 0};
-      if (gather) gather_rows(p, t, t.row0 + 4 * lane, rtok);
-      const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
-      const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
-      const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
-      for (int kb = 0; kb < p.kb_per_split; ++kb) {
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-          if (lane == 0) {
-            atomicOr(p.status, kStatusProducerTimeout);
-            *abort_flag = 1;
-          }
-          goto producer_done;
-        }
-        uint8_t* xs = smem + stage * C::STAGE_BYTES;
-        uint8_t* ws = xs + X_BYTES;
-        uint8_t* w8 = ws + W_BYTES;
-        const int k0 = (t.kb0 + kb) * BK;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full_bar[stage], xbytes + wbytes);
-          if (WS) {
-            for (int b = 0; b < nbox_x; ++b)
-              tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
-          } else if (!gather) {
-            tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
-          }
-          if (W8) {
-            if (KIND == GATEUP) {
-              load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
-              load_w(w8 + W8_BYTES / 2, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
-            } else {
-              load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
-              load_w(w8 + W8_BYTES / 2, &tm_w0, &full_bar[stage], t.n0 + 128, k0, t.e);
+    auto produce = [&](auto gather_tag) {
+      constexpr bool G = decltype(gather_tag)::value;
+      int stage = 0;
+      uint32_t phase = 0;
+      Tile t;
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+        int32_t rtok[4] = {0, 0, 0, 0};
+        if (G) gather_rows(p, t, t.row0 + 4 * lane, rtok);
+        const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
+        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
+        const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
+        for (int kb = 0; kb < p.kb_per_split; ++kb) {
+          int ok = 1;
+          if (!G || lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
+          if (G) ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) {
+            if (!G || lane == 0) {
+              atomicOr(p.status, kStatusProducerTimeout);
+              *abort_flag = 1;
             }
-          } else {
-            if (KIND == GATEUP) {
-              // chunks 0,1: gate columns n0..n0+127; chunks 2,3: up columns n0..n0+127
-              load_w(ws + 0 * WCHUNK, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
-              load_w(ws + 1 * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64, k0, t.e);
-              load_w(ws + 2 * WCHUNK, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
-              load_w(ws + 3 * WCHUNK, &tm_w1, &full_bar[stage], t.n0 + 64, k0, t.e);
+            return;
+          }
+          uint8_t* xs = smem + stage * C::STAGE_BYTES;
+          uint8_t* ws = xs + X_BYTES;
+          uint8_t* w8 = ws + W_BYTES;
+          const int k0 = (t.kb0 + kb) * BK;
+          if (!G || lane == 0) {
+            mbar_arrive_expect_tx(&full_bar[stage], xbytes + wbytes);
+            if (WS) {
+              for (int b = 0; b < nbox_x; ++b)
+                tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
+            } else if (!G) {
+              tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
+            }
+            if (W8) {
+              if (KIND == GATEUP) {
+                load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+                load_w(w8 + W8_BYTES / 2, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
+              } else {
+                load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+                load_w(w8 + W8_BYTES / 2, &tm_w0, &full_bar[stage], t.n0 + 128, k0, t.e);
+              }
             } else {
-              for (int j = 0; j < 4; ++j)
-                load_w(ws + j * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64 * j, k0, t.e);
+              if (KIND == GATEUP) {
+                // chunks 0,1: gate columns n0..n0+127; chunks 2,3: up columns n0..n0+127
+                load_w(ws + 0 * WCHUNK, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
+                load_w(ws + 1 * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64, k0, t.e);
+                load_w(ws + 2 * WCHUNK, &tm_w1, &full_bar[stage], t.n0, k0, t.e);
+                load_w(ws + 3 * WCHUNK, &tm_w1, &full_bar[stage], t.n0 + 64, k0, t.e);
+              } else {
+                for (int j = 0; j < 4; ++j)
+                  load_w(ws + j * WCHUNK, &tm_w0, &full_bar[stage], t.n0 + 64 * j, k0, t.e);
+              }
             }
           }
-        }
-        __syncwarp();  // the barrier is armed before any lane's gather can complete on it
-        // Lane l fills A rows 4l .. 4l+3 (512 B, 128-B swizzled like one tall box).
-        if (gather) tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
+          if (G) {
+            __syncwarp();  // the barrier is armed before any lane's gather can complete on it
+            // Lane l fills A rows 4l .. 4l+3 (512 B, 128-B swizzled like one tall box).
+            tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
+    };
+    if (!WS && KIND == GATEUP && p.row_token != nullptr) {
+      if constexpr (!WS && KIND == GATEUP) produce(std::true_type{});
+    } else if (lane == 0) {
+      produce(std::false_type{});
     }
-  producer_done:;
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {

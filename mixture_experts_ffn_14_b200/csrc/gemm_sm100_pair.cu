@@ -26,6 +26,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "gemm_common.cuh"
 
@@ -127,75 +128,86 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
     // ------------------------------------------------------------ producer --
     // Lane 0 waits for a free stage, arms the barrier and loads the weight box
     // (and the activation box of materialised rows); with the row gather each
-    // of the 32 lanes also loads four of this CTA's 128 token rows from x.
-    const bool gather = KIND == GATEUP && p.row_token != nullptr;
-    int stage = 0;
-    uint32_t phase = 0;
-    Tile t;
-    for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
-      const int row = t.row0 + BM * static_cast<int>(rank);
-      int32_t rtok[4] = {0, 0, 0, 0};
-      if (gather) gather_rows(p, t, row + 4 * lane, rtok);
-      // GATEUP: the even CTA holds the gate columns, the odd one the up
-      // columns (accumulator columns 0..127 / 128..255). DOWN: 128 columns each.
-      const CUtensorMap* wmap = (KIND == GATEUP && rank == 1) ? &tm_w1 : &tm_w0;
-      const int n = KIND == GATEUP ? t.n0 : t.n0 + 128 * static_cast<int>(rank);
-      for (int kb = 0; kb < p.kb_per_split; ++kb) {
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-          if (lane == 0) {
-            atomicOr(p.status, kStatusProducerTimeout);
-            *abort_flag = 1;
+    // of the 32 lanes also loads four of this CTA's 128 token rows from x. The
+    // two variants are compiled separately so that the plain one stays lane 0
+    // alone with no warp-synchronous step.
+    auto produce = [&](auto gather_tag) {
+      constexpr bool G = decltype(gather_tag)::value;
+      int stage = 0;
+      uint32_t phase = 0;
+      Tile t;
+      for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
+        const int row = t.row0 + BM * static_cast<int>(rank);
+        int32_t rtok[4] = {0, 0, 0, 0};
+        if (G) gather_rows(p, t, row + 4 * lane, rtok);
+        // GATEUP: the even CTA holds the gate columns, the odd one the up
+        // columns (accumulator columns 0..127 / 128..255). DOWN: 128 columns each.
+        const CUtensorMap* wmap = (KIND == GATEUP && rank == 1) ? &tm_w1 : &tm_w0;
+        const int n = KIND == GATEUP ? t.n0 : t.n0 + 128 * static_cast<int>(rank);
+        for (int kb = 0; kb < p.kb_per_split; ++kb) {
+          int ok = 1;
+          if (!G || lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs) && !*abort_flag;
+          if (G) ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) {
+            if (!G || lane == 0) {
+              atomicOr(p.status, kStatusProducerTimeout);
+              *abort_flag = 1;
+            }
+            return;
           }
-          goto producer_done;
-        }
-        {
           uint8_t* xs = smem + stage * C::STAGE_BYTES;
           uint8_t* ws = xs + X_BYTES;
           uint8_t* w8 = ws + PW_BYTES;
           const int k0 = (t.kb0 + kb) * BK;
           if (W8) {
-            if (lane == 0) {
+            if (!G || lane == 0) {
               mbar_arrive_expect_tx(&full_bar[stage], X_BYTES + PW8_BYTES);
-              if (!gather) tma_load_2d(xs, &tm_x, &full_bar[stage], k0, row);
+              if (!G) tma_load_2d(xs, &tm_x, &full_bar[stage], k0, row);
               tma_load_3d(w8, wmap, &full_bar[stage], n, k0, t.e);
             }
-            __syncwarp();  // armed before any lane's gather can complete on it
-            if (gather) tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+            if (G) {
+              __syncwarp();  // armed before any lane's gather can complete on it
+              tma_gather4(xs + lane * 512, &tm_x, &full_bar[stage], k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+            }
           } else {
             const uint32_t bar0 = mapa_shared(&full_bar[stage], 0);
-            if (lane == 0) {
+            if (!G || lane == 0) {
               if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (X_BYTES + PW_BYTES));
-              if (!gather) tma_load_2d_pair(xs, &tm_x, bar0, k0, row);
+              if (!G) tma_load_2d_pair(xs, &tm_x, bar0, k0, row);
               tma_load_3d_pair(ws, wmap, bar0, n, k0, t.e);
               tma_load_3d_pair(ws + WCHUNK, wmap, bar0, n + 64, k0, t.e);
             }
-            __syncwarp();
-            if (gather) tma_gather4_pair(xs + lane * 512, &tm_x, bar0, k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+            if (G) {
+              __syncwarp();
+              tma_gather4_pair(xs + lane * 512, &tm_x, bar0, k0, rtok[0], rtok[1], rtok[2], rtok[3]);
+            }
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
+      }
+      // Drain: every stage's last release (an arrive sent by the pair's MMA
+      // commit) has landed before this CTA may exit.
+      if (!G || lane == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs)) {
+            atomicOr(p.status, kStatusProducerTimeout);
+            break;
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
+    };
+    if (KIND == GATEUP && p.row_token != nullptr) {
+      if constexpr (KIND == GATEUP) produce(std::true_type{});
+    } else if (lane == 0) {
+      produce(std::false_type{});
     }
-    // Drain: every stage's last release (an arrive sent by the pair's MMA
-    // commit) has landed before this CTA may exit.
-    if (lane == 0) {
-      for (int i = 0; i < STAGES; ++i) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, kWaitLimitNs)) {
-          atomicOr(p.status, kStatusProducerTimeout);
-          break;
-        }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-  producer_done:;
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0 && rank == 0) {
