@@ -70,19 +70,26 @@ def peaks():
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi samples every 100 ms; only those whose own timestamp falls
-    inside the `with` block count (its output reaches the pipe in blocks, so the
-    arrival time of a line says nothing)."""
+    """SM clock, power and clock-event reasons sampled DURING the `with` block.
 
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML (read-only queries) every 20 ms from a background thread; if NVML is
+    unavailable, nvidia-smi every 100 ms, keeping the samples whose own
+    timestamp falls inside the block."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+    SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, torch_dev):
         import torch
 
-        self.proc = None
-        self.lines = []
+        self.samples = []        # (sm_mhz, sm_max_mhz, power_w, {reason names})
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
         self._t0 = self._t1 = None
         try:
             pr = torch.cuda.get_device_properties(torch_dev)
@@ -90,63 +97,94 @@ class ClockSampler:
         except Exception:
             self.bus = None
 
-    def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+    # ---- NVML
+    def _nvml_loop(self, nv, h):
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(smax), pw, {n for n, m in self.REASONS if bits & m}))
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def _start_nvml(self):
+        import threading
+
+        import pynvml as nv
+
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByPciBusId(self.bus.encode()) if self.bus else nv.nvmlDeviceGetHandleByIndex(0)
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+        self._thread.start()
+        self.source = "nvml"
+
+    # ---- nvidia-smi fallback
+    def _start_smi(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.bus:
             cmd += ["-i", self.bus]
+        self._proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        time.sleep(0.5)  # let it start sampling before the region opens
+        self.source = "nvidia-smi"
+
+    def _finish_smi(self):
+        time.sleep(0.15)
+        self._proc.terminate()
         try:
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            time.sleep(0.5)  # let it start sampling before the region opens
+            out, _ = self._proc.communicate(timeout=5)
         except Exception:
-            self.proc = None
+            self._proc.kill()
+            out = ""
+        stamped = []
+        for ln in out.splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                smp = (float(parts[2]), float(parts[3]), float(parts[4]),
+                       {n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                           "sw_power_cap"), parts[6:10]) if v.lower() == "active"})
+            except ValueError:
+                continue
+            stamped.append((t, smp))
+        inside = [smp for t, smp in stamped if self._t0 <= t <= self._t1]
+        if not inside and stamped:  # region shorter than a sample period: the nearest sample
+            mid = 0.5 * (self._t0 + self._t1)
+            inside = [min(stamped, key=lambda ts: abs(ts[0] - mid))[1]]
+        self.samples = inside
+
+    def __enter__(self):
+        try:
+            self._start_nvml()
+        except Exception:
+            try:
+                self._start_smi()
+            except Exception:
+                self.source = None
         self._t0 = time.time()
         return self
 
     def __exit__(self, *exc):
         self._t1 = time.time()
-        if self.proc is None:
-            return
-        time.sleep(0.15)  # one more sample period
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out = ""
-        stamped = []
-        for ln in out.splitlines():
-            ts = ln.split(",", 1)[0].strip()
-            try:
-                t = datetime.datetime.strptime(ts, "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                continue
-            stamped.append((t, ln.split(",", 1)[1]))
-        inside = [ln for t, ln in stamped if self._t0 <= t <= self._t1]
-        if not inside and stamped:  # region shorter than a sample period: the nearest sample
-            mid = 0.5 * (self._t0 + self._t1)
-            inside = [min(stamped, key=lambda tl: abs(tl[0] - mid))[1]]
-        self.lines = inside
+        if self.source == "nvml":
+            self._stop.set()
+            self._thread.join(timeout=5)
+        elif self.source == "nvidia-smi":
+            self._finish_smi()
 
     def summary(self):
-        sm, smax, power, reasons = [], None, [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power) if power else None}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [x[0] for x in self.samples]
+        reasons = set().union(*(x[3] for x in self.samples))
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.samples[-1][1], "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(x[2] for x in self.samples),
+                "power_w_median": statistics.median(x[2] for x in self.samples), "source": self.source}
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -382,7 +420,8 @@ def main():
         "roofline": roofline,
         "gpu_launches": launches_per_step(wl, a.path) * K,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
-                   "power_w_max": clocks.get("power_w_max"), "samples": clocks.get("samples")},
+                   "power_w_max": clocks.get("power_w_max"), "power_w_median": clocks.get("power_w_median"),
+                   "samples": clocks.get("samples"), "source": clocks.get("source")},
         "wall_s_timed_region": round(wall, 3),
     }
     if e2e:
@@ -399,13 +438,16 @@ def main():
 
 
 def recorded_traffic(wl):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu record,
-    or None when the workload differs or the GEMM sources changed since."""
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu record of
+    this workload, or None when there is none or the GEMM sources changed since."""
     import hashlib
     import re
 
-    path = os.path.join(ROOT, "profiles", "gemm_traffic_prefill_T4096.md")
-    if not os.path.exists(path) or (wl.name, wl.T, wl.d, wl.f) != ("prefill", 4096, 6144, 32768):
+    records = {("prefill", 4096, 6144, 32768): "gemm_traffic_prefill_T4096.md",
+               ("decode", 64, 6144, 32768): "gemm_traffic_decode_T64.md"}
+    name = records.get((wl.name, wl.T, wl.d, wl.f))
+    path = os.path.join(ROOT, "profiles", name) if name else None
+    if not path or not os.path.exists(path):
         return None
     m = re.search(r"```json\n(.*?)\n```", open(path).read(), re.S)
     if not m:
@@ -437,7 +479,7 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks):
         dn = touched * d * f * esz / (dn_ms / 1e3) / 1e9
         return {"bound": "hbm", "kernel": "moe_expert_gemm_kernel<GATEUP, WEIGHT_STREAM>",
                 "achieved": round(gu, 1), "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gu / pk["hbm_gbs"], 4),
-                "traffic": None, "peak_source": f"{pk['source']} HBM copy",
+                "traffic": recorded_traffic(wl), "peak_source": f"{pk['source']} HBM copy",
                 "algorithmic_per_launch": gu_bytes,
                 "down_gemm": {"achieved": round(dn, 1), "frac": round(dn / pk["hbm_gbs"], 4)}}
     gu = 8 * T * d * f / (gu_ms / 1e3) / 1e12
@@ -451,44 +493,89 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks):
 
 
 def run_e2e(a, moe, inp, run, out, flush, dist, dev, world, flops):
-    """Same metric through the public API with the batch in pinned host memory:
-    every timed step copies x in and the result out."""
+    """Same metric through the public API with every batch in pinned host memory.
+
+    Each timed step copies its x in (host -> device), runs the layer and copies
+    its result out (device -> host). Two device buffers per side let the copy of
+    step i+1's input and of step i-1's output run on their own streams while
+    step i computes, as a serving loop would; the region spans all K steps and
+    ends when the last output has reached the host. The serial form (copy in,
+    compute, copy out, one after the other) is reported beside it."""
     import torch
 
     T, d = inp["x"].shape
     K = a.steps
     x_host = inp["x"].cpu().pin_memory()
-    out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
+    out_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xs = [torch.empty_like(inp["x"]) for _ in range(2)]
+    outs = [torch.empty((T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     plain = "s_gate" not in inp and "router_bias" not in inp
+    main = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    used = [torch.cuda.Event() for _ in range(2)]      # step done with xs[b] / outs[b]
+    fetched = [torch.cuda.Event() for _ in range(2)]   # outs[b] has reached the host
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
+    def forward(x_dev, o):
         if plain:
-            moe.moe_forward(x_dev, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out)
+            moe.moe_forward(x_dev, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], o, stream=main)
         else:
-            run(x_dev, out)
-        out_host.copy_(out, non_blocking=True)
+            run(x_dev, o)
 
-    for _ in range(a.warmup):
-        flush.zero_()
-        e2e_step()
+    def step(i):
+        b = i % 2
+        ready = torch.cuda.Event()
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(used[b])
+            xs[b].copy_(x_host, non_blocking=True)
+            ready.record(h2d)
+        main.wait_event(ready)
+        main.wait_event(fetched[b])
+        forward(xs[b], outs[b])
+        used[b].record(main)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(used[b])
+            out_host[b].copy_(outs[b], non_blocking=True)
+            fetched[b].record(d2h)
+
+    for i in range(a.warmup):
+        step(i)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(main)
+    h2d.wait_event(t0)
+    d2h.wait_event(t0)
+    for i in range(K):
+        step(i)
+    main.wait_stream(h2d)
+    main.wait_stream(d2h)
+    t1.record(main)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
+
+    # Serial form: each step's copies and compute back to back on one stream.
     e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     for i in range(K):
         flush.zero_()
-        e_s[i].record()
-        e2e_step()
-        e_e[i].record()
+        e_s[i].record(main)
+        xs[0].copy_(x_host, non_blocking=True)
+        forward(xs[0], outs[0])
+        out_host[0].copy_(outs[0], non_blocking=True)
+        e_e[i].record(main)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dist, dev)
+    serial_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dist, dev)
     return {"value": round(world * K * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+            "ms_per_step": round(e2e_ms / K, 4),
             "api": ("moe_forward (library workspace)" if plain else "moe_forward_ex")
-                   + ", pinned host x -> device -> pinned host out"}
+                   + ", pinned host x -> device -> pinned host out",
+            "overlap": "double-buffered: copies of step i+1's input and step i-1's output on their own streams "
+                       "during step i; region from the first copy-in to the last copy-out",
+            "l2": "not flushed: every step streams the full weight set (> 70x L2)",
+            "serial_value": round(world * K * flops / (serial_ms / 1e3) / 1e12, 2),
+            "serial_ms_per_step": round(serial_ms / K, 4)}
 
 
 def run_decode(a, moe, W, wl, inp, dev, pk):
