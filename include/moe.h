@@ -74,7 +74,11 @@ typedef enum {
 typedef enum {
   MOE_F32 = 0,         /* fp32 activations and weights, fp32 arithmetic        */
   MOE_BF16 = 1,        /* bf16 activations and weights, fp32 accumulation      */
-  MOE_BF16_INT8W = 2   /* bf16 activations, int8 weights + bf16 channel scales */
+  MOE_BF16_INT8W = 2   /* bf16 activations, int8 weights + bf16 channel scales;
+                          the expert GEMMs run on fp16 operands: int8 -> fp16 is
+                          exact, bf16 activations -> fp16 is exact for normal
+                          values below 65504 in magnitude, and the GeGLU
+                          intermediate is kept in fp16 (range |h| < 65504)     */
 } moe_dtype_t;
 
 /* Activation on the gate branch of every expert. */
@@ -141,7 +145,8 @@ typedef struct {
                                   dispatch stage (default); 1: they gather their gate/up
                                   operand rows from x with TMA row gathers (no copy; slower
                                   on B200, where four-row gathers cannot feed the MMA).
-                                  The weight-stream form always reads the copy.           */
+                                  The weight-stream form always reads the copy;
+                                  MOE_BF16_INT8W returns MOE_ERR_UNSUPPORTED with 1.      */
 } moe_options_t;
 
 /* Optional outputs for inspection; each is a device pointer or NULL.
@@ -153,8 +158,9 @@ typedef struct {
   int32_t* offsets;    /* [E+1]  exclusive prefix of counts                 */
   int32_t* perm_token; /* [2T]   token of each permuted row                 */
   int32_t* perm_slot;  /* [2T]   slot (0/1) of each permuted row            */
-  void* h;             /* [2T, f] x-dtype: GELU(x.Wg)*(x.Wu) per permuted row;
-                          when set, the kernels write the intermediate here   */
+  void* h;             /* [2T, f] GELU(x.Wg)*(x.Wu) per permuted row: x-dtype,
+                          but fp16 for MOE_BF16_INT8W; when set, the kernels
+                          write the intermediate here                         */
 } moe_debug_t;
 
 /* Forward pass with a library-owned workspace: one cache per device, grown

@@ -6,6 +6,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -154,24 +155,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Four int8 values (one 32-bit word) -> four bf16 (two 32-bit words), exact:
-// flip the sign bit to get q + 128 in [1, 255], place it in the low mantissa
-// bits of 2^23, subtract 2^23 + 128 in fp32. An integer |q| <= 127 uses at most
-// the top 7 fraction bits of the fp32 result, so its low 16 bits are zero and
-// its high half is exactly the bf16 value: pack the high halves with a byte
-// permute (no rounding step needed).
-__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t v;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));  // upper half from the first source
+  return v;
+}
+
+// Four int8 values (one 32-bit word) -> four fp16 (two 32-bit words), exact:
+// flip the sign bit to get q + 128 in [0, 255], make it the low mantissa byte of
+// fp16 1024 (0x6400: exponent 2^10, unit mantissa step), so each half is
+// 1024 + q + 128, then one packed subtraction of 1152 leaves q. Both operands lie
+// in [1024, 2048), so the difference is exact, and every |q| <= 128 is an fp16.
+__device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
   const uint32_t u = w ^ 0x80808080u;
-  const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
-  const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
-  const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
-  const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
-  lo = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
-  hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x7632);
+  const uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);  // halves 0x64:b0, 0x64:b1
+  const uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);  // halves 0x64:b2, 0x64:b3
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x64806480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x64806480u));
 }
 
 // Convert 16-byte int8 segment `seg` of a staging area made of [64 K][128 N]
-// int8 boxes into the bf16 weight tile: box b covers bf16 chunks 2b and 2b+1,
+// int8 boxes into the fp16 weight tile: box b covers fp16 chunks 2b and 2b+1,
 // each [64 K][64 N] with the 128-B swizzle (16-B unit u of row k is stored at
 // unit u ^ (k % 8)).
 __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t* wtile, int seg) {
@@ -181,12 +185,12 @@ __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t*
   const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (BK * 128) + k * 128 + c16 * 16);
   const int col = c16 * 16;        // 0..112
   const int chunk = box * 2 + (col >> 6);
-  const int u = (col & 63) >> 3;   // 16-B unit of the bf16 row (even)
+  const int u = (col & 63) >> 3;   // 16-B unit of the fp16 row (even)
   uint32_t o[8];
-  i8x4_to_bf16x4(src.x, o[0], o[1]);
-  i8x4_to_bf16x4(src.y, o[2], o[3]);
-  i8x4_to_bf16x4(src.z, o[4], o[5]);
-  i8x4_to_bf16x4(src.w, o[6], o[7]);
+  i8x4_to_f16x4(src.x, o[0], o[1]);
+  i8x4_to_f16x4(src.y, o[2], o[3]);
+  i8x4_to_f16x4(src.z, o[4], o[5]);
+  i8x4_to_f16x4(src.w, o[6], o[7]);
   uint8_t* rowp = wtile + chunk * WCHUNK + k * 128;
   *reinterpret_cast<uint4*>(rowp + ((u ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -194,7 +198,7 @@ __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t*
 
 // Token-tile epilogue of one epilogue warp: TMEM lane = token row r (0..127 of
 // this CTA's rows starting at permuted row `row_base`), 256 accumulator
-// columns. GATEUP: columns 0..127 gate, 128..255 up -> bf16 H[row, n0 + c].
+// columns. GATEUP: columns 0..127 gate, 128..255 up -> H[row, n0 + c] (bf16; fp16 with int8 weights).
 // DOWN: 256 output columns -> fp32 Y[split, row, n0 + c] = acc * gate[row].
 template <int KIND, bool W8>
 __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile& t, uint32_t tbase, int r,
@@ -202,7 +206,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
   const bool valid = r < nvalid;
   const int64_t row = row_base + r;
   if (KIND == GATEUP) {
-    __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
+    uint16_t* hout = static_cast<uint16_t*>(p.out);
 #pragma unroll 1
     for (int c = 0; c < 128; c += 32) {
       uint32_t g[32], u[32];
@@ -219,7 +223,9 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
           u0 *= __bfloat162float(p.s1[sc]);
           u1 *= __bfloat162float(p.s1[sc + 1]);
         }
-        packed[j / 2] = pack_bf16x2(act_f32(g0, p.act) * u0, act_f32(g1, p.act) * u1);
+        // int8 weights run the MMAs on fp16 operands, so H is stored as fp16 there.
+        const float h0 = act_f32(g0, p.act) * u0, h1 = act_f32(g1, p.act) * u1;
+        packed[j / 2] = W8 ? pack_f16x2(h0, h1) : pack_bf16x2(h0, h1);
       }
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);

@@ -209,7 +209,10 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
         const uint32_t ntok = WS ? ((t.rows + 15) / 16) * 16 : 0;
-        const uint32_t idesc = WS ? idesc_bf16_f32(128, ntok, 1, 0) : idesc_bf16_f32(128, 256, 0, 1);
+        // int8 weights are converted to fp16 (exact), and the activations they
+        // meet are fp16 too: one operand type per MMA.
+        const uint32_t idesc = W8 ? (WS ? idesc_f16_f32(128, ntok, 1, 0) : idesc_f16_f32(128, 256, 0, 1))
+                                  : (WS ? idesc_bf16_f32(128, ntok, 1, 0) : idesc_bf16_f32(128, 256, 0, 1));
         for (int kb = 0; kb < p.kb_per_split; ++kb) {
           uint64_t* ready = W8 ? &conv_bar[stage] : &full_bar[stage];
           if (!mbar_wait(ready, phase, kWaitLimitNs) || *abort_flag) {
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
         // Weight-stream: TMEM lane = output column, TMEM column = token.
         const int ntok = ((t.rows + 15) / 16) * 16;
         if (KIND == GATEUP) {
-          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(p.out);
+          uint16_t* hout = static_cast<uint16_t*>(p.out);  // bf16, or fp16 with int8 weights
           const int n = t.n0 + 32 * q + lane;
           float sg = 1.0f, su = 1.0f;
           if (W8) {
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             for (int j = 0; j < 32; ++j) {
               if (c + j < t.rows) {
                 const float h = act_f32(__uint_as_float(g[j]) * sg, p.act) * (__uint_as_float(u[j]) * su);
-                hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] = __float2bfloat16_rn(h);
+                hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] =
+                    W8 ? __half_as_ushort(__float2half_rn(h)) : __bfloat16_as_ushort(__float2bfloat16_rn(h));
               }
             }
           }
@@ -324,8 +328,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       }
     }
   } else if (W8 && warp >= 8) {
-    // ----------------------------------------------- int8 -> bf16 convert --
-    // Staging: two int8 boxes [64 K][128 N] (row = 128 B). Target: four bf16
+    // ----------------------------------------------- int8 -> fp16 convert --
+    // Staging: two int8 boxes [64 K][128 N] (row = 128 B). Target: four fp16
     // chunks [64 K][64 N] with the 128-B swizzle (16-B unit u of row k stored at
     // unit u ^ (k % 8)).
     const int ct = threadIdx.x - 256;  // 0 .. CONVERT_THREADS-1
@@ -380,7 +384,8 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
     const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(gather ? a.x_rows : a.rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
     const uint32_t box[2] = {BK, static_cast<uint32_t>(gather ? 1 : WS ? XBOX_ROWS_WS : BM)};
-    if (!encode_tensor_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, dims, strides, box,
+    if (!encode_tensor_map(&tm_x, W8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x,
+                           dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }

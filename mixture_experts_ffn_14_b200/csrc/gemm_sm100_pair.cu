@@ -215,7 +215,8 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      const uint32_t idesc = idesc_bf16_f32(PAIR_ROWS, 256, 0, 1);
+      // int8 weights: fp16 operands on both sides (exact conversion).
+      const uint32_t idesc = W8 ? idesc_f16_f32(PAIR_ROWS, 256, 0, 1) : idesc_bf16_f32(PAIR_ROWS, 256, 0, 1);
       Tile t;
       for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
         if (!mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
@@ -370,7 +371,8 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
     const uint64_t dims[2] = {static_cast<uint64_t>(a.K), static_cast<uint64_t>(gather ? a.x_rows : a.rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(a.K) * 2};
     const uint32_t box[2] = {BK, static_cast<uint32_t>(gather ? 1 : BM)};
-    if (!encode_tensor_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, dims, strides, box,
+    if (!encode_tensor_map(&tm_x, W8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x,
+                           dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }

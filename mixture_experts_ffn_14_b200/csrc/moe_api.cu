@@ -276,6 +276,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE) return MOE_ERR_INVALID_ARG;
   if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
   if (o->row_gather != 0 && o->row_gather != 1) return MOE_ERR_INVALID_ARG;
+  // The int8-weight GEMMs take fp16 activations from the dispatch copy; a row
+  // gather would feed them x's bf16 rows.
+  if (o->row_gather == 1 && a->dtype == MOE_BF16_INT8W) return MOE_ERR_UNSUPPORTED;
   if (o->router_bias && !aligned16(o->router_bias)) return MOE_ERR_MISALIGNED;
   const bool h_ext = dbg && dbg->h;
   if (h_ext && !aligned16(dbg->h)) return MOE_ERR_MISALIGNED;

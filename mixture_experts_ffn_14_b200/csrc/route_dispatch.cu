@@ -219,11 +219,23 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(
   if (threadIdx.x < kE) hist[blk * kE + threadIdx.x] = cnt[threadIdx.x];
 }
 
+// Eight bf16 (one 16-byte vector) -> eight fp16, round to nearest even.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));
+  return r;
+}
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+}
+
 // Same 32-token range per CTA as the router. Each CTA sums the per-CTA
 // histograms to find where its tokens land (no cross-CTA waiting), ranks its
 // tokens per expert with warp ballots (token order = stable), writes the
 // permutation arrays and copies the x rows to their permuted positions.
-template <typename TX>
+// F16: the copy converts bf16 rows to fp16 (round to nearest even), for the
+// int8-weight GEMMs, whose MMAs run on fp16 operands.
+template <typename TX, bool F16 = false>
 __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     const TX* __restrict__ x, int64_t T, int64_t d, int64_t nblk, const int32_t* __restrict__ idx,
     const float* __restrict__ gates, const int32_t* __restrict__ hist, int32_t* __restrict__ counts,
@@ -339,7 +351,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u)
-      if (o[u] >= 0) dst[o[u]] = v[u];
+      if (o[u] >= 0) dst[o[u]] = F16 ? bf16x8_to_f16x8(v[u]) : v[u];
   }
 }
 
@@ -512,6 +524,10 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
     moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(
         static_cast<const float*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
         slot_pos, gate_perm, static_cast<float*>(xp));
+  else if (dtype == MOE_BF16_INT8W)
+    moe_dispatch_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp));
   else
     moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,

@@ -171,6 +171,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // a_mn / b_mn: 1 when that operand is MN-major in shared memory.
+// Same with fp16 A and B (kind::f16 takes one operand type for both: the
+// format fields of A and B are always set together).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
+  return (1u << 4)          // D format: f32
+         | (0u << 7)        // A format: f16
+         | (0u << 10)       // B format: f16
+         | (a_mn << 15)     // A major
+         | (b_mn << 16)     // B major
+         | ((N >> 3) << 17) // N / 8
+         | ((M >> 4) << 24);// M / 16
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
   return (1u << 4)          // D format: f32
          | (1u << 7)        // A format: bf16

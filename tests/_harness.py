@@ -41,8 +41,9 @@ def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, activation=moe.MOE_ACT_GELU_TA
         "perm_token": torch.empty(2 * T, dtype=torch.int32, device=dev),
         "perm_slot": torch.empty(2 * T, dtype=torch.int32, device=dev),
     }
-    if want_h:
-        dbg["h"] = torch.empty((2 * T, f), dtype=x.dtype, device=dev)
+    if want_h:   # the int8-weight path keeps its intermediate in fp16
+        h_dtype = torch.float16 if inp["w_gate"].dtype == torch.int8 else x.dtype
+        dbg["h"] = torch.empty((2 * T, f), dtype=h_dtype, device=dev)
     scales = (inp["s_gate"], inp["s_up"], inp["s_down"]) if "s_gate" in inp else None
     moe.moe_forward_ex(x, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws, scales=scales,
                        router_bias=inp.get("router_bias"), activation=activation, path=path, down_splits=down_splits,
