@@ -44,14 +44,21 @@ constexpr int W_BYTES = 4 * WCHUNK;     // 32 KB: four [64 K x 64 N] chunks
 constexpr int W8_BYTES = BK * 256;      // 16 KB int8 staging: two [64 K x 128 N] boxes
 constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
 
+// Shared memory. bf16 weights: STAGES slots of [X tile | W tile] (48 KB).
+// int8 weights: two rings, so that more of the shared memory holds loads in
+// flight: STAGES slots of [X tile | int8 W staging] (32 KB) filled by TMA, and
+// CSTAGES slots of converted fp16 W tiles (32 KB) that the converter warps fill
+// one stage ahead of the MMA.
 template <bool W8>
 struct Cfg {
-  static constexpr int STAGES = W8 ? 3 : 4;
-  static constexpr int STAGE_BYTES = X_BYTES + W_BYTES + (W8 ? W8_BYTES : 0);
+  static constexpr int STAGES = W8 ? 5 : 4;
+  static constexpr int SLOT_BYTES = X_BYTES + (W8 ? W8_BYTES : W_BYTES);
+  static constexpr int CSTAGES = W8 ? 2 : 0;
+  static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : 256;
   static constexpr int BAR_BYTES = 1024;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
 
 template <int KIND, bool WS, bool W8>
@@ -63,11 +70,13 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-B swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* bar_area = smem + STAGES * C::STAGE_BYTES;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
-  uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* conv_bar = empty_bar + STAGES;
-  uint64_t* tfull_bar = conv_bar + STAGES;
+  uint8_t* conv_area = smem + STAGES * C::SLOT_BYTES;  // int8: converted W ring
+  uint8_t* bar_area = smem + C::RING_BYTES;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);  // TMA slot filled
+  uint64_t* empty_bar = full_bar + STAGES;                      // TMA slot free again
+  uint64_t* cfull_bar = empty_bar + STAGES;                     // converted W slot ready
+  uint64_t* cempty_bar = cfull_bar + 2;                         // converted W slot free again
+  uint64_t* tfull_bar = cempty_bar + 2;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -81,8 +90,12 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-      mbar_init(&conv_bar[s], C::CONVERT_THREADS);
+      // int8: freed by the MMA commit (X read) and every converter thread (W8 read)
+      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_THREADS : 1);
+    }
+    for (int c = 0; c < C::CSTAGES; ++c) {
+      mbar_init(&cfull_bar[c], C::CONVERT_THREADS);
+      mbar_init(&cempty_bar[c], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -142,9 +155,9 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             }
             return;
           }
-          uint8_t* xs = smem + stage * C::STAGE_BYTES;
-          uint8_t* ws = xs + X_BYTES;
-          uint8_t* w8 = ws + W_BYTES;
+          uint8_t* xs = smem + stage * C::SLOT_BYTES;
+          uint8_t* ws = xs + X_BYTES;  // bf16 W tile, or the int8 staging (W8)
+          uint8_t* w8 = ws;
           const int k0 = (t.kb0 + kb) * BK;
           if (!G || lane == 0) {
             mbar_arrive_expect_tx(&full_bar[stage], xbytes + wbytes);
@@ -197,6 +210,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int cstage = 0;       // int8: converted W ring
+      uint32_t cphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       Tile t;
@@ -214,15 +229,17 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
         const uint32_t idesc = W8 ? (WS ? idesc_f16_f32(128, ntok, 1, 0) : idesc_f16_f32(128, 256, 0, 1))
                                   : (WS ? idesc_bf16_f32(128, ntok, 1, 0) : idesc_bf16_f32(128, 256, 0, 1));
         for (int kb = 0; kb < p.kb_per_split; ++kb) {
-          uint64_t* ready = W8 ? &conv_bar[stage] : &full_bar[stage];
-          if (!mbar_wait(ready, phase, kWaitLimitNs) || *abort_flag) {
+          // int8: the converted W tile, then the X tile of the same K block (its
+          // TMA slot completed before the converters could start on it).
+          if ((W8 && !mbar_wait(&cfull_bar[cstage], cphase, kWaitLimitNs)) ||
+              !mbar_wait(&full_bar[stage], phase, kWaitLimitNs) || *abort_flag) {
             atomicOr(p.status, kStatusMmaTimeout);
             *abort_flag = 1;
             goto mma_done;
           }
           tc_fence_after();
-          const uint32_t xs = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t ws = xs + X_BYTES;
+          const uint32_t xs = smem_u32(smem + stage * C::SLOT_BYTES);
+          const uint32_t ws = W8 ? smem_u32(conv_area + cstage * W_BYTES) : xs + X_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < BK / 16; ++k16) {
             const uint32_t accum = (kb | k16) != 0;
@@ -242,6 +259,13 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             }
           }
           umma_commit(&empty_bar[stage]);
+          if (W8) {
+            umma_commit(&cempty_bar[cstage]);
+            if (++cstage == C::CSTAGES) {
+              cstage = 0;
+              cphase ^= 1;
+            }
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -329,33 +353,40 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     }
   } else if (W8 && warp >= 8) {
     // ----------------------------------------------- int8 -> fp16 convert --
-    // Staging: two int8 boxes [64 K][128 N] (row = 128 B). Target: four fp16
-    // chunks [64 K][64 N] with the 128-B swizzle (16-B unit u of row k stored at
-    // unit u ^ (k % 8)).
+    // Staging: two int8 boxes [64 K][128 N] (row = 128 B) in TMA slot `stage`.
+    // Target: converted slot `cstage`, four fp16 chunks [64 K][64 N] with the
+    // 128-B swizzle (16-B unit u of row k stored at unit u ^ (k % 8)).
     const int ct = threadIdx.x - 256;  // 0 .. CONVERT_THREADS-1
     int stage = 0;
     uint32_t phase = 0;
+    int cstage = 0;
+    uint32_t cphase = 0;
     Tile t;
     for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
-        if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) || *abort_flag) {
+        if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) ||
+            !mbar_wait(&cempty_bar[cstage], cphase ^ 1, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusConvertTimeout);
           *abort_flag = 1;
           goto convert_done;
         }
         {
-          uint8_t* xs = smem + stage * C::STAGE_BYTES;
-          uint8_t* ws = xs + X_BYTES;
-          const uint8_t* w8 = ws + W_BYTES;
+          const uint8_t* w8 = smem + stage * C::SLOT_BYTES + X_BYTES;
+          uint8_t* wc = conv_area + cstage * W_BYTES;
 #pragma unroll
           for (int it = 0; it < 1024 / C::CONVERT_THREADS; ++it)
-            convert_int8_segment(w8, ws, ct + C::CONVERT_THREADS * it);
+            convert_int8_segment(w8, wc, ct + C::CONVERT_THREADS * it);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&conv_bar[stage]);
+        fence_proxy_async_smem();      // converted tile visible to the MMA (async proxy)
+        mbar_arrive(&empty_bar[stage]);  // this thread is done reading the staging slot
+        mbar_arrive(&cfull_bar[cstage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
+        }
+        if (++cstage == C::CSTAGES) {
+          cstage = 0;
+          cphase ^= 1;
         }
       }
     }
