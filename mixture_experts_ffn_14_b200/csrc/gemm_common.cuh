@@ -178,10 +178,22 @@ __device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
 // int8 boxes into the fp16 weight tile: box b covers fp16 chunks 2b and 2b+1,
 // each [64 K][64 N] with the 128-B swizzle (16-B unit u of row k is stored at
 // unit u ^ (k % 8)).
+//
+// Segment order. 16-byte shared-memory accesses are served eight threads at a
+// time, and each group of eight must touch eight different 16-B bank groups to
+// take one pass. Within every 16 consecutive segments (one row pair k, k+1) the
+// first eight take columns 0-3 of row k and 4-7 of row k+1, the next eight the
+// rest: the loads (unswizzled staging, unit = c16) then hit units 0..7, and the
+// two swizzled stores of a group land on units (u ^ k) with u = 0, 2, 4, 6 for
+// the even row and on the odd units for the odd row, again all eight distinct.
+// (Row-major order, eight groups of one row, wrote every unit twice: one per
+// 64-column chunk.)
 __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t* wtile, int seg) {
   const int box = seg >> 9;        // 512 segments per box
-  const int k = (seg >> 3) & 63;   // row
-  const int c16 = seg & 7;         // 16-column group in the 128-wide row
+  const int g = seg & 511;
+  const int i = g & 7;
+  const int k = 2 * (g >> 4) + (i >> 2);          // row
+  const int c16 = i ^ (((g >> 3) & 1) << 2);      // 16-column group in the 128-wide row
   const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (BK * 128) + k * 128 + c16 * 16);
   const int col = c16 * 16;        // 0..112
   const int chunk = box * 2 + (col >> 6);
