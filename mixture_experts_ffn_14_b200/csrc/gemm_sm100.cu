@@ -56,6 +56,7 @@ struct Cfg {
   static constexpr int CSTAGES = W8 ? 2 : 0;
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
+  static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
   static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : 256;
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
@@ -90,11 +91,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      // int8: freed by the MMA commit (X read) and every converter thread (W8 read)
-      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_THREADS : 1);
+      // int8: freed by the MMA commit (X read) and every converter warp (W8 read)
+      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_WARPS : 1);
     }
     for (int c = 0; c < C::CSTAGES; ++c) {
-      mbar_init(&cfull_bar[c], C::CONVERT_THREADS);
+      mbar_init(&cfull_bar[c], C::CONVERT_WARPS);
       mbar_init(&cempty_bar[c], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -377,9 +378,12 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           for (int it = 0; it < 1024 / C::CONVERT_THREADS; ++it)
             convert_int8_segment(w8, wc, ct + C::CONVERT_THREADS * it);
         }
-        fence_proxy_async_smem();      // converted tile visible to the MMA (async proxy)
-        mbar_arrive(&empty_bar[stage]);  // this thread is done reading the staging slot
-        mbar_arrive(&cfull_bar[cstage]);
+        fence_proxy_async_smem();  // this thread's converted stores visible to the async proxy
+        __syncwarp();              // ... and the whole warp's, before one arrive per warp
+        if (lane == 0) {
+          mbar_arrive(&empty_bar[stage]);  // staging slot read
+          mbar_arrive(&cfull_bar[cstage]);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
