@@ -188,24 +188,46 @@ __device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
 // the even row and on the odd units for the odd row, again all eight distinct.
 // (Row-major order, eight groups of one row, wrote every unit twice: one per
 // 64-column chunk.)
-__device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t* wtile, int seg) {
-  const int box = seg >> 9;        // 512 segments per box
+// Bounded wait taken by a whole warp: every lane waits, and the warp goes on
+// only if every lane saw the phase complete and no role has aborted, so the
+// warp-synchronous instructions after it (tcgen05.ld, __syncwarp) never run on
+// part of a warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, kWaitLimitNs) && !*abort_flag;
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct SegPos {
+  int box, k, c16;  // int8 box (0, 1), row 0..63, 16-column group 0..7
+};
+
+__device__ __forceinline__ SegPos seg_pos(int seg) {
   const int g = seg & 511;
   const int i = g & 7;
-  const int k = 2 * (g >> 4) + (i >> 2);          // row
-  const int c16 = i ^ (((g >> 3) & 1) << 2);      // 16-column group in the 128-wide row
-  const uint4 src = *reinterpret_cast<const uint4*>(w8 + box * (BK * 128) + k * 128 + c16 * 16);
-  const int col = c16 * 16;        // 0..112
-  const int chunk = box * 2 + (col >> 6);
-  const int u = (col & 63) >> 3;   // 16-B unit of the fp16 row (even)
+  return {seg >> 9, 2 * (g >> 4) + (i >> 2), i ^ (((g >> 3) & 1) << 2)};
+}
+
+// Sixteen int8 weights of segment `sp` (row k, columns 16*c16 .. +15 of box b)
+// -> fp16, stored into the weight tile: box b covers fp16 chunks 2b and 2b+1.
+__device__ __forceinline__ void convert_store_segment(uint4 src, uint8_t* wtile, SegPos sp) {
+  const int col = sp.c16 * 16;        // 0..112
+  const int chunk = sp.box * 2 + (col >> 6);
+  const int u = (col & 63) >> 3;      // 16-B unit of the fp16 row (even)
   uint32_t o[8];
   i8x4_to_f16x4(src.x, o[0], o[1]);
   i8x4_to_f16x4(src.y, o[2], o[3]);
   i8x4_to_f16x4(src.z, o[4], o[5]);
   i8x4_to_f16x4(src.w, o[6], o[7]);
-  uint8_t* rowp = wtile + chunk * WCHUNK + k * 128;
-  *reinterpret_cast<uint4*>(rowp + ((u ^ (k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-  *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  uint8_t* rowp = wtile + chunk * WCHUNK + sp.k * 128;
+  *reinterpret_cast<uint4*>(rowp + ((u ^ (sp.k & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (sp.k & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Same, reading the segment from an int8 staging area of [64 K][128 N] boxes.
+__device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t* wtile, int seg) {
+  const SegPos sp = seg_pos(seg);
+  const uint4 src = *reinterpret_cast<const uint4*>(w8 + sp.box * (BK * 128) + sp.k * 128 + sp.c16 * 16);
+  convert_store_segment(src, wtile, sp);
 }
 
 // Token-tile epilogue of one epilogue warp: TMEM lane = token row r (0..127 of

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     uint32_t acc_phase = 0;
     Tile t;
     for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, kWaitLimitNs) || *abort_flag) {
+      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
         break;
@@ -365,8 +365,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     Tile t;
     for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
-        if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) ||
-            !mbar_wait(&cempty_bar[cstage], cphase ^ 1, kWaitLimitNs) || *abort_flag) {
+        if (!warp_wait(&full_bar[stage], phase, abort_flag) || !warp_wait(&cempty_bar[cstage], cphase ^ 1, abort_flag)) {
           atomicOr(p.status, kStatusConvertTimeout);
           *abort_flag = 1;
           goto convert_done;

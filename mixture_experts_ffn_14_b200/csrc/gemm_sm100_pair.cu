@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
     uint32_t acc_phase = 0;
     Tile t;
     for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, kWaitLimitNs) || *abort_flag) {
+      if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
         break;
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
     Tile t;
     for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
-        if (!mbar_wait(&full_bar[stage], phase, kWaitLimitNs) || *abort_flag) {
+        if (!warp_wait(&full_bar[stage], phase, abort_flag)) {
           atomicOr(p.status, kStatusConvertTimeout);
           *abort_flag = 1;
           goto convert_done;
