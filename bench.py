@@ -596,6 +596,23 @@ def run_decode(a, moe, W, wl, inp, dev, pk):
     step_ms, stage_ms = timed_steps(run, xd, outd, K, None)
     d_ms = statistics.mean(step_ms)
     wbytes = touched * 3 * d * f * 2
+    # The same step captured once in a CUDA graph and replayed (no per-launch
+    # host work, no stage events): what a serving loop that replays graphs sees.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run(xd, outd)
+    torch.cuda.synchronize()
+    for _ in range(a.warmup):
+        graph.replay()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    g0.record()
+    for _ in range(K):
+        graph.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    g_ms = g0.elapsed_time(g1) / K
+    del graph
     return {"workload": f"grok1-decode T={Td} d={d} f={f} bf16 (same weights)",
             "ms_per_step": round(d_ms, 4), "experts_touched": touched,
             "hbm_gbs": round(wbytes / (d_ms / 1e3) / 1e9, 1),
@@ -603,6 +620,7 @@ def run_decode(a, moe, W, wl, inp, dev, pk):
             "gate_up_gbs": round(touched * 2 * d * f * 2 / (stage_ms["gate_up_gemm"] / 1e3) / 1e9, 1),
             "down_gbs": round(touched * d * f * 2 / (stage_ms["down_gemm"] / 1e3) / 1e9, 1),
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "graph_ms_per_step": round(g_ms, 4), "graph_hbm_gbs": round(wbytes / (g_ms / 1e3) / 1e9, 1),
             "peak_gbs": pk["hbm_gbs"], "bytes_per_step": wbytes}
 
 
