@@ -437,10 +437,26 @@ def main():
     return 0
 
 
+def gemm_code_hash(sources):
+    """SHA-256 of the GEMM sources with comments and trailing blanks removed: a
+    traffic record stays valid while the code is the one it was captured on."""
+    import hashlib
+    import re
+
+    h = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, src)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
+    return h.hexdigest()
+
+
 def recorded_traffic(wl):
     """DRAM bytes per launch of the gate/up GEMM from the committed ncu record of
-    this workload, or None when there is none or the GEMM sources changed since."""
-    import hashlib
+    this workload, or None when there is none or the GEMM code changed since."""
     import re
 
     records = {("prefill", 4096, 6144, 32768): "gemm_traffic_prefill_T4096.md",
@@ -453,11 +469,7 @@ def recorded_traffic(wl):
     if not m:
         return None
     rec = json.loads(m.group(1))
-    h = hashlib.sha256()
-    for src in rec["gemm_sources"]:
-        with open(os.path.join(ROOT, src), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest() != rec["gemm_source_sha256"]:
+    if gemm_code_hash(rec["gemm_sources"]) != rec["gemm_code_sha256"]:
         return None
     k = rec["kernels"]["gate_up"]
     return k["dram_read_bytes"] + k["dram_write_bytes"]

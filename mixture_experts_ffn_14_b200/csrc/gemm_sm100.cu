@@ -11,12 +11,15 @@
 //   warp 0      TMA producer: activation tile + weight tile per 64-deep K stage
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one thread)
 //   warps 4..7  epilogue: tcgen05.ld from TMEM, activation / gate / scale, global stores
-//   warps 8..15 (int8 weights only) convert the int8 stage to bf16 in shared memory
+//   warps 8..15 (int8 weights only) convert the int8 stage to fp16 in shared memory
 //               (two warps per SM sub-partition, so one hides the other's latency)
 //
 // Shared memory per stage: X tile [128 rows x 64 K] bf16, K-major, 128-B swizzle
 // (16 KB) and W tile = four chunks [64 K x 64 N] bf16, N(MN)-major, 128-B swizzle
 // (32 KB); weights are used in the caller's [E, K, N] layout without a repack.
+// int8 weights: the same tiles in fp16 (activations converted by the dispatch
+// stage, weights by the converter warps), with the int8 staging in the TMA ring
+// and the converted W tiles in a ring of their own (see Cfg).
 //
 // Orientation:
 //   TOKEN_TILE    MMA M = 128 token rows (A = X, K-major), N = 256 weight columns

@@ -17,7 +17,7 @@
 // tcgen05.commit multicast to the barriers of both CTAs. Epilogue warps of
 // both CTAs arrive on the even CTA's accumulator-empty barrier.
 // int8 weights: each CTA's loads complete on its own full barrier; its
-// converter warps turn its int8 half into bf16 and arrive on the even CTA's
+// converter warps turn its int8 half into fp16 and arrive on the even CTA's
 // converted barrier, on which the MMA thread waits.
 // Every wait is bounded; a timeout records a status bit and unwinds.
 #include <cuda.h>
