@@ -315,9 +315,11 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 def launches_per_step(wl, path):
     """Kernels of ours per step: router, dispatch, two GEMMs, combine; with the
     automatic token-tile choice on bf16 weights each GEMM launches both forms
-    (the one not chosen returns at once)."""
+    (the one not chosen returns at once); above 1024 router blocks (T > 32768)
+    a histogram scan runs before the dispatch."""
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
-    return 5 + (2 if both else 0)
+    scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
+    return 5 + (2 if both else 0) + (1 if scan else 0)
 
 
 # ---------------------------------------------------------------- main --

@@ -244,6 +244,7 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   L.idx = take(sizeof(int32_t) * rows);
   L.gates = take(sizeof(float) * rows);
   L.hist = take(sizeof(int32_t) * L.nblk * kE);
+  L.hist_pre = take(sizeof(int32_t) * (L.nblk + 1) * kE);  // block prefixes + totals (many blocks)
   L.logits_part = L.router_slices > 1 ? take(sizeof(float) * L.router_slices * T * kE) : 0;
   L.counts = take(sizeof(int32_t) * kE);
   L.offsets = take(sizeof(int32_t) * (kE + 1));
@@ -292,6 +293,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
   float* gates = reinterpret_cast<float*>(ws + L.gates);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* hist_pre = reinterpret_cast<int32_t*>(ws + L.hist_pre);
   int32_t* arrivals = reinterpret_cast<int32_t*>(ws + L.arrivals);
   float* logits_part = L.router_slices > 1 ? reinterpret_cast<float*>(ws + L.logits_part) : nullptr;
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
@@ -322,8 +324,8 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, L.router_slices,
                         logits_part, arrivals, idx, gates, hist, stream));
   MOE_TRY(mark(1));
-  MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
-                          slot_pos, gate_perm, xp, stream));
+  MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, hist_pre, counts, offsets, perm_token,
+                          perm_slot, slot_pos, gate_perm, xp, stream));
   MOE_TRY(mark(2));
   if (a->dtype == MOE_F32) {
     MOE_TRY(launch_f32_gateup(static_cast<const float*>(xp), static_cast<const float*>(a->w_gate),

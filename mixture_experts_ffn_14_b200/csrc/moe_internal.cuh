@@ -28,8 +28,8 @@ enum : uint32_t {
 
 // Byte offsets of the regions of one call's workspace (each 256-aligned).
 struct WorkspaceLayout {
-  size_t status, arrivals, idx, gates, hist, logits_part, counts, offsets, perm_token, perm_slot, slot_pos,
-      gate_perm;
+  size_t status, arrivals, idx, gates, hist, hist_pre, logits_part, counts, offsets, perm_token, perm_slot,
+      slot_pos, gate_perm;
   size_t xp, h, y, total;
   int64_t nblk;      // router / dispatch CTAs
   int32_t splits;    // split-K factor of the down projection
@@ -56,10 +56,15 @@ cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_route
                           int64_t d, int32_t renormalize, int32_t slices, float* partial, int32_t* arrivals,
                           int32_t* idx, float* gates, int32_t* hist, cudaStream_t s);
 
+// Dispatch. With more than kDispatchSumBlocks router blocks a one-CTA scan of
+// the block histograms runs first, into hist_pre [nblk * E + E] (prefixes, then
+// totals); with fewer, each dispatch CTA sums the histograms it needs itself.
+constexpr int64_t kDispatchSumBlocks = 1024;
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
-                            const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
-                            int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
-                            float* gate_perm, void* xp, cudaStream_t s);  // xp == nullptr: no row copy
+                            const int32_t* idx, const float* gates, const int32_t* hist, int32_t* hist_pre,
+                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
+                            int32_t* slot_pos, float* gate_perm, void* xp,
+                            cudaStream_t s);  // xp == nullptr: no row copy
 
 // out[t] = residual[t] + norm(y0 + y1); residual and norm_weight may be NULL.
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,

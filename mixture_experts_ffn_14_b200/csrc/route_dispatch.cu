@@ -219,6 +219,70 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(
   if (threadIdx.x < kE) hist[blk * kE + threadIdx.x] = cnt[threadIdx.x];
 }
 
+// Exclusive prefix over router blocks of the per-block expert histograms, and
+// their totals, for batches with many blocks (one CTA of 1024 threads: thread i
+// owns a contiguous run of blocks, sums it, the CTA scans the 1024 run sums per
+// expert, and each thread writes its run's prefixes). Linear in the blocks, so
+// the dispatch CTAs read their offsets instead of summing all predecessors.
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) moe_hist_scan_kernel(const int32_t* __restrict__ hist, int64_t nblk,
+                                                                     int32_t* __restrict__ pre,
+                                                                     int32_t* __restrict__ tot) {
+  __shared__ int wsum[kE][kScanThreads / 32];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int64_t per = (nblk + kScanThreads - 1) / kScanThreads;
+  const int64_t b0 = min(nblk, tid * per), b1 = min(nblk, b0 + per);
+  int run[kE];
+#pragma unroll
+  for (int e = 0; e < kE; ++e) run[e] = 0;
+  for (int64_t b = b0; b < b1; ++b) {
+    const int4 lo = *reinterpret_cast<const int4*>(hist + b * kE);
+    const int4 hi = *reinterpret_cast<const int4*>(hist + b * kE + 4);
+    run[0] += lo.x; run[1] += lo.y; run[2] += lo.z; run[3] += lo.w;
+    run[4] += hi.x; run[5] += hi.y; run[6] += hi.z; run[7] += hi.w;
+  }
+  // Exclusive scan of the run sums over the CTA, per expert.
+  int excl[kE];
+#pragma unroll
+  for (int e = 0; e < kE; ++e) {
+    int v = run[e];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    excl[e] = v - run[e];                       // exclusive within the warp
+    if (lane == 31) wsum[e][warp] = v;          // warp total
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+      const int w = wsum[e][lane];
+      int v = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      wsum[e][lane] = v - w;                    // exclusive over warps
+      if (lane == 31) tot[e] = v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < kE; ++e) excl[e] += wsum[e][warp];
+  for (int64_t b = b0; b < b1; ++b) {
+    const int4 lo = *reinterpret_cast<const int4*>(hist + b * kE);
+    const int4 hi = *reinterpret_cast<const int4*>(hist + b * kE + 4);
+    *reinterpret_cast<int4*>(pre + b * kE) = make_int4(excl[0], excl[1], excl[2], excl[3]);
+    *reinterpret_cast<int4*>(pre + b * kE + 4) = make_int4(excl[4], excl[5], excl[6], excl[7]);
+    excl[0] += lo.x; excl[1] += lo.y; excl[2] += lo.z; excl[3] += lo.w;
+    excl[4] += hi.x; excl[5] += hi.y; excl[6] += hi.z; excl[7] += hi.w;
+  }
+}
+
 // Eight bf16 (one 16-byte vector) -> eight fp16, round to nearest even.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   uint32_t r;
@@ -240,7 +304,8 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     const TX* __restrict__ x, int64_t T, int64_t d, int64_t nblk, const int32_t* __restrict__ idx,
     const float* __restrict__ gates, const int32_t* __restrict__ hist, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
-    int32_t* __restrict__ slot_pos, float* __restrict__ gate_perm, TX* __restrict__ xp) {
+    int32_t* __restrict__ slot_pos, float* __restrict__ gate_perm, TX* __restrict__ xp,
+    const int32_t* __restrict__ hist_pre, const int32_t* __restrict__ hist_tot) {
   // blockIdx.y splits the row gather of the block across gridDim.y CTAs; all of
   // them rank the block's tokens (cheap), the first one writes the permutation.
   __shared__ int red[8][2 * kE];
@@ -249,15 +314,27 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t blk = blockIdx.x;
 
+  // This block's slots start, per expert, after those of all earlier blocks:
+  // read from the scan (many blocks) or summed here (few blocks, no extra launch).
   int tot[kE], pre[kE];
 #pragma unroll
   for (int e = 0; e < kE; ++e) tot[e] = pre[e] = 0;
-  for (int64_t c = threadIdx.x; c < nblk; c += blockDim.x) {
+  if (hist_pre != nullptr) {
+    if (threadIdx.x == 0) {
 #pragma unroll
-    for (int e = 0; e < kE; ++e) {
-      const int v = hist[c * kE + e];
-      tot[e] += v;
-      if (c < blk) pre[e] += v;
+      for (int e = 0; e < kE; ++e) {
+        tot[e] = hist_tot[e];
+        pre[e] = hist_pre[blk * kE + e];
+      }
+    }
+  } else {
+    for (int64_t c = threadIdx.x; c < nblk; c += blockDim.x) {
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        const int v = hist[c * kE + e];
+        tot[e] += v;
+        if (c < blk) pre[e] += v;
+      }
     }
   }
 #pragma unroll
@@ -513,9 +590,20 @@ cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_route
 }
 
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
-                            const int32_t* idx, const float* gates, const int32_t* hist, int32_t* counts,
-                            int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos,
-                            float* gate_perm, void* xp, cudaStream_t s) {
+                            const int32_t* idx, const float* gates, const int32_t* hist, int32_t* hist_pre,
+                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
+                            int32_t* slot_pos, float* gate_perm, void* xp, cudaStream_t s) {
+  // Many router blocks: scan their histograms once (hist_pre holds nblk * E
+  // prefixes followed by E totals); few: each dispatch CTA sums them itself.
+  const int32_t* pre = nullptr;
+  const int32_t* tot = nullptr;
+  if (nblk > kDispatchSumBlocks) {
+    moe_hist_scan_kernel<<<1, kScanThreads, 0, s>>>(hist, nblk, hist_pre, hist_pre + nblk * kE);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    pre = hist_pre;
+    tot = hist_pre + nblk * kE;
+  }
   // Extra CTAs along y only split the row gather; without Xp one suffices.
   const int64_t g =
       xp ? std::min<int64_t>(16, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk)) : 1;
@@ -523,15 +611,15 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
   if (dtype == MOE_F32)
     moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(
         static_cast<const float*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
-        slot_pos, gate_perm, static_cast<float*>(xp));
+        slot_pos, gate_perm, static_cast<float*>(xp), pre, tot);
   else if (dtype == MOE_BF16_INT8W)
     moe_dispatch_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
-        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp));
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot);
   else
     moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
-        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp));
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot);
   return cudaGetLastError();
 }
 

@@ -58,3 +58,55 @@ def test_full_shape_decode_both_paths_agree():
     assert np.array_equal(a["idx"], b["idx"])
     err = np.abs(a["out"] - b["out"])
     assert (err <= 1e-2 + 2e-2 * np.abs(b["out"])).all()
+
+
+def test_max_token_count_large_offsets():
+    # T = 2^24, the largest batch the library accepts, at d = 256, f = 128: x and
+    # the permuted copy hold 2^32 and 2^33 elements, H 2^32, the fp32 down
+    # partials 2^33, so every index past 2^31 must be 64-bit. Routing and outputs
+    # are checked against the oracle on sampled tokens (the first and last
+    # included); counts, offsets and the permutation over all 2^25 slots against
+    # their definition (stable sort by (expert, token)), vectorised in numpy.
+    import mixture_experts_ffn_14_b200 as moe
+    import oracle
+    from _harness import assert_close, expected_routing, np64
+
+    T, d, f = 1 << 24, 256, 128
+    w = W.Workload("max_tokens", T, d, f, dtype="bf16", seed=97)
+    inp = W.make_torch(w, DEV)
+    ws = torch.empty(moe.moe_workspace_size(T, d, f), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(inp["x"])
+    dbg = {"idx": torch.empty((T, 2), dtype=torch.int32, device=DEV),
+           "gates": torch.empty((T, 2), dtype=torch.float32, device=DEV),
+           "counts": torch.empty(8, dtype=torch.int32, device=DEV),
+           "offsets": torch.empty(9, dtype=torch.int32, device=DEV),
+           "perm_token": torch.empty(2 * T, dtype=torch.int32, device=DEV),
+           "perm_slot": torch.empty(2 * T, dtype=torch.int32, device=DEV)}
+    moe.moe_forward_ex(inp["x"], inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws, debug=dbg)
+    torch.cuda.synchronize()
+    st, code = moe.moe_device_status(ws)
+    assert st == 0 and code == 0
+    del ws
+
+    idx = dbg["idx"].cpu().numpy()
+    counts = dbg["counts"].cpu().numpy().astype(np.int64)
+    offsets = dbg["offsets"].cpu().numpy().astype(np.int64)
+    assert (idx[:, 0] != idx[:, 1]).all() and idx.min() >= 0 and idx.max() < 8
+    assert (counts == np.bincount(idx.ravel(), minlength=8)).all() and counts.sum() == 2 * T
+    assert (offsets == np.concatenate([[0], np.cumsum(counts)])).all()
+    key = idx.ravel().astype(np.int64) * T + np.repeat(np.arange(T, dtype=np.int64), 2)
+    order = np.argsort(key, kind="stable")
+    assert (dbg["perm_token"].cpu().numpy() == order // 2).all()
+    assert (dbg["perm_slot"].cpu().numpy() == order % 2).all()
+    del key, order
+
+    tok = sample_tokens(T, n=48, seed=5)
+    sel = torch.as_tensor(tok, device=DEV)
+    x64 = np64(inp["x"][sel])
+    wr64 = np64(inp["w_router"])
+    routing, _ = expected_routing(x64, wr64, None, idx[tok])
+    assert (routing["idx"] == idx[tok]).all()
+    assert np.max(np.abs(dbg["gates"][sel].cpu().numpy() - routing["gates"])) <= 2e-6
+    experts = tuple(np64(inp[n]) for n in ("w_gate", "w_up", "w_down"))
+    ref = oracle.forward_sparse(x64, wr64, experts, routing=routing)["out"]
+    assert_close(np64(out[sel]), ref, "out")

@@ -113,6 +113,18 @@ def test_row_gather_skewed_with_empty_experts():
     full_check(inp, run_gpu(inp, row_gather=True))
 
 
+@pytest.mark.parametrize("T", [32768, 32800, 40000])
+def test_dispatch_scan_threshold(T):
+    # Up to 1024 router blocks (T = 32768) each dispatch CTA sums the block
+    # histograms itself; above, a one-CTA scan computes the block offsets first.
+    # Full dispatch against the oracle on both sides of the threshold; outputs on
+    # a sample of tokens (first and last included).
+    inp = small_bf16(T, d=256, f=128, seed=41)
+    rng = np.random.default_rng(T)
+    tok = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 64, replace=False)]))
+    full_check(inp, run_gpu(inp, want_h=False), tokens=tok, check_h=False)
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3])
 def test_bf16_weight_stream_split_k(splits):
     inp = small_bf16(90, d=256, f=384)

@@ -53,3 +53,6 @@ def test_launch_count_rule():
     assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 5
     assert bench.launches_per_step(W.WORKLOADS["int8"], "auto") == 5
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "token_tile") == 5
+    import dataclasses
+    big = dataclasses.replace(W.WORKLOADS["prefill"], T=40000)   # > 1024 router blocks: + scan
+    assert bench.launches_per_step(big, "auto") == 8
