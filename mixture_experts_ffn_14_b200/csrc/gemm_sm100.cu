@@ -51,12 +51,12 @@ constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
 // int8 weights: two rings, so that more of the shared memory holds loads in
 // flight: STAGES slots of [X tile | int8 W staging] (32 KB) filled by TMA, and
 // CSTAGES slots of converted fp16 W tiles (32 KB) that the converter warps fill
-// one stage ahead of the MMA.
+// up to two stages ahead of the MMA (4 + 3 measured ~3 % faster than 5 + 2).
 template <bool W8>
 struct Cfg {
-  static constexpr int STAGES = W8 ? 5 : 4;
+  static constexpr int STAGES = 4;
   static constexpr int SLOT_BYTES = X_BYTES + (W8 ? W8_BYTES : W_BYTES);
-  static constexpr int CSTAGES = W8 ? 2 : 0;
+  static constexpr int CSTAGES = W8 ? 3 : 0;
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
@@ -64,6 +64,10 @@ struct Cfg {
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
+constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ring
+static_assert(Cfg<true>::CSTAGES <= kMaxCStages, "converted-W ring deeper than its barrier slots");
+static_assert((2 * Cfg<true>::STAGES + 2 * kMaxCStages + 4) * 8 + 16 + sizeof(SharedSched) <= Cfg<true>::BAR_BYTES,
+              "barrier area too small");
 
 template <int KIND, bool WS, bool W8>
 __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
@@ -79,8 +83,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);  // TMA slot filled
   uint64_t* empty_bar = full_bar + STAGES;                      // TMA slot free again
   uint64_t* cfull_bar = empty_bar + STAGES;                     // converted W slot ready
-  uint64_t* cempty_bar = cfull_bar + 2;                         // converted W slot free again
-  uint64_t* tfull_bar = cempty_bar + 2;
+  uint64_t* cempty_bar = cfull_bar + kMaxCStages;               // converted W slot free again
+  uint64_t* tfull_bar = cempty_bar + kMaxCStages;
   uint64_t* tempty_bar = tfull_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
