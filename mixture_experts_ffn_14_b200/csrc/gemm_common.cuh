@@ -44,6 +44,7 @@ struct Params {
   int32_t act;           // moe_activation_t of the gate branch
   int32_t select;        // kRunAlways, or run only if the pair / single form is preferred
   int32_t sm_count;      // SMs of the device (same value for both token-tile kernels)
+  int32_t* tile_counter; // CTA-pair kernel, bf16 weights: tiles handed out in order (zero on entry)
   uint32_t* status;
 };
 

@@ -447,6 +447,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.offsets = a.offsets;
   p.gate_perm = a.gate_perm;
   p.row_token = (!WS && KIND == GATEUP) ? a.row_token : nullptr;
+  p.tile_counter = nullptr;  // static tile order
   p.s0 = a.s0;
   p.s1 = a.s1;
   p.out = a.out;

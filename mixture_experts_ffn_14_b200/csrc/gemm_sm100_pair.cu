@@ -37,6 +37,20 @@ constexpr int PAIR_ROWS = 2 * BM;      // 256 token rows per pair tile
 constexpr int PW_BYTES = 2 * WCHUNK;   // 16 KB: this CTA's 128 weight columns
 constexpr int PW8_BYTES = BK * 128;    // 8 KB: one int8 box [64 K x 128 N]
 
+// Tile order. With bf16 weights the pair kernel hands out tiles dynamically:
+// the even CTA's producer takes the next tile id from a global counter when it
+// starts a tile, and writes it into slot i % kTileQ of both CTAs' tile-id
+// queues; every other role reads its tiles from its own CTA's queue in the same
+// order and frees the slot on the even CTA's qempty barrier. Consecutive tile
+// ids are the row tiles that share one weight tile, and they go to the pairs that
+// become free together, so those pairs read the weight tile from L2 close in
+// time. (With static round-robin order the pairs that share a weight tile change
+// every wave and drift apart, and the weights are fetched from DRAM again.)
+// int8 weights keep the static order: their converter warps would be a third
+// kind of reader.
+constexpr int kTileQ = 4;            // producer leads the epilogue by at most 3 tiles
+constexpr int kTileQConsumers = 10;  // odd producer, MMA thread, 4 epilogue warps x 2 CTAs
+
 template <bool W8>
 struct PairCfg {
   static constexpr int STAGES = W8 ? 5 : 6;
@@ -84,9 +98,12 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
   uint64_t* conv_bar = empty_bar + STAGES;
   uint64_t* tfull_bar = conv_bar + STAGES;
   uint64_t* tempty_bar = tfull_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  uint64_t* qfull_bar = tempty_bar + 2;      // tile-id queue slot written
+  uint64_t* qempty_bar = qfull_bar + kTileQ;  // tile-id queue slot read by every role (even CTA's)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty_bar + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   SharedSched* sched = reinterpret_cast<SharedSched*>(tmem_slot + 4);
+  volatile int* tile_q = reinterpret_cast<volatile int*>(sched + 1);
 
   if (skip_launch(p)) return;  // the other token-tile form takes this call
 
@@ -106,6 +123,10 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 2 * 4);  // four epilogue warps in each CTA
     }
+    for (int i = 0; i < kTileQ; ++i) {
+      mbar_init(&qfull_bar[i], 1);
+      mbar_init(&qempty_bar[i], kTileQConsumers);
+    }
     *abort_flag = 0;
     build_sched(*sched, p, PAIR_ROWS);
     fence_mbar_init();
@@ -124,6 +145,41 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // ---- tile order (see kTileQ). Queue operations return the tile id, -1 when
+  // no tile is left, -2 when a wait timed out.
+  const bool dyn = !W8 && p.tile_counter != nullptr;
+  const int ntiles = sched->pre[kE];
+  auto q_fill = [&](int i) -> int {  // even CTA's producer
+    const int slot = i % kTileQ;
+    const uint32_t ph = (i / kTileQ) & 1;
+    if (!mbar_wait_cluster(&qempty_bar[slot], ph ^ 1, kWaitLimitNs) || *abort_flag) return -2;
+    const int t = atomicAdd(p.tile_counter, 1);
+    const int tile = t < ntiles ? t : -1;
+    tile_q[slot] = tile;
+    st_shared_cluster_u32(mapa_shared(const_cast<int*>(&tile_q[slot]), 1), static_cast<uint32_t>(tile));
+    mbar_arrive(&qfull_bar[slot]);
+    mbar_arrive_cluster(mapa_shared(&qfull_bar[slot], 1));
+    return tile;
+  };
+  auto q_take = [&](int i) -> int {  // one thread of any other role
+    const int slot = i % kTileQ;
+    const uint32_t ph = (i / kTileQ) & 1;
+    if (!mbar_wait_cluster(&qfull_bar[slot], ph, kWaitLimitNs) || *abort_flag) return -2;
+    const int tile = tile_q[slot];
+    mbar_arrive_cluster(mapa_shared(&qempty_bar[slot], 0));
+    return tile;
+  };
+  auto q_take_warp = [&](int i) -> int {  // a whole epilogue warp, one arrive
+    const int slot = i % kTileQ;
+    const uint32_t ph = (i / kTileQ) & 1;
+    const bool ok = mbar_wait_cluster(&qfull_bar[slot], ph, kWaitLimitNs) && !*abort_flag;
+    if (!__all_sync(0xffffffffu, ok)) return -2;
+    const int tile = tile_q[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(mapa_shared(&qempty_bar[slot], 0));
+    return tile;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     // Lane 0 waits for a free stage, arms the barrier and loads the weight box
@@ -136,7 +192,20 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       Tile t;
-      for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
+      for (int i = 0;; ++i) {
+        int tile = pair + i * npairs;
+        if (dyn) {
+          if (!G || lane == 0) tile = rank == 0 ? q_fill(i) : q_take(i);
+          if (G) tile = __shfl_sync(0xffffffffu, tile, 0);
+          if (tile == -2) {
+            if (!G || lane == 0) {
+              atomicOr(p.status, kStatusProducerTimeout);
+              *abort_flag = 1;
+            }
+            return;
+          }
+        }
+        if (tile < 0 || !decode_tile(*sched, p, tile, PAIR_ROWS, t)) break;
         const int row = t.row0 + BM * static_cast<int>(rank);
         int32_t rtok[4] = {0, 0, 0, 0};
         if (G) gather_rows(p, t, row + 4 * lane, rtok);
@@ -218,7 +287,14 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
       // int8 weights: fp16 operands on both sides (exact conversion).
       const uint32_t idesc = W8 ? idesc_f16_f32(PAIR_ROWS, 256, 0, 1) : idesc_bf16_f32(PAIR_ROWS, 256, 0, 1);
       Tile t;
-      for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
+      for (int i = 0;; ++i) {
+        const int tile = dyn ? q_take(i) : pair + i * npairs;
+        if (tile == -2) {
+          atomicOr(p.status, kStatusMmaTimeout);
+          *abort_flag = 1;
+          goto mma_done;
+        }
+        if (tile < 0 || !decode_tile(*sched, p, tile, PAIR_ROWS, t)) break;
         if (!mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusMmaTimeout);
           *abort_flag = 1;
@@ -267,7 +343,14 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
-    for (int tile = pair; decode_tile(*sched, p, tile, PAIR_ROWS, t); tile += npairs) {
+    for (int i = 0;; ++i) {
+      const int tile = dyn ? q_take_warp(i) : pair + i * npairs;
+      if (tile == -2) {
+        atomicOr(p.status, kStatusEpilogueTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      if (tile < 0 || !decode_tile(*sched, p, tile, PAIR_ROWS, t)) break;
       if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
@@ -393,6 +476,7 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   p.offsets = a.offsets;
   p.gate_perm = a.gate_perm;
   p.row_token = KIND == GATEUP ? a.row_token : nullptr;
+  p.tile_counter = W8 ? nullptr : a.tile_counter;
   p.s0 = a.s0;
   p.s1 = a.s1;
   p.out = a.out;

@@ -290,6 +290,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  // Tile counters of the two CTA-pair GEMM launches, in the status slot (zeroed
+  // with it below).
+  int32_t* tile_counters = reinterpret_cast<int32_t*>(ws + L.status + 16);
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
   float* gates = reinterpret_cast<float*>(ws + L.gates);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
@@ -356,6 +359,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.int8_weights = w8;
     g.weight_stream = L.weight_stream;
     g.status = status;
+    g.tile_counter = tile_counters;
     // Token tiles: with MOE_PATH_AUTO both forms are launched and the kernels
     // pick one of them on the device from the expert counts (the other returns
     // at once); TOKEN_TILE / TOKEN_TILE_SINGLE force one form.
@@ -390,6 +394,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g2.K = static_cast<int32_t>(f);
     g2.N = static_cast<int32_t>(d);
     g2.splits = L.splits;
+    g2.tile_counter = tile_counters + 1;
     MOE_TRY(launch_gemm(g2, true));
   }
   MOE_TRY(mark(4));

@@ -98,6 +98,7 @@ struct TcGemmArgs {
   bool int8_weights;
   bool weight_stream;
   int32_t select;           // 0: always run; 1 / 2: run only if the pair / single token-tile form is preferred
+  int32_t* tile_counter;    // pair form: zeroed int that hands out tiles in order, or nullptr (static order)
   uint32_t* status;
 };
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
