@@ -169,7 +169,7 @@ bool use_weight_stream(int64_t T, moe_path_t path) {
 // and few (rows/128 x d/256), so the last partial wave can idle most SMs. For
 // balanced loads (each expert pads on average half a tile) estimate, per split
 // factor s, the time of the waves of whichever tile form the kernels will pick
-// (single-CTA 128-row tiles, or CTA-pair 256-row tiles at a 3 % discount), plus
+// (single-CTA 128-row tiles, or CTA-pair 256-row tiles at a 7 % discount), plus
 // 2.3 % of the unsplit work per extra split for the fp32 partial sums that are
 // written and read again (their bytes relative to the GEMM time at d, f).
 int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested, bool allow_single,
@@ -188,7 +188,7 @@ int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t r
     if (!valid(s)) continue;
     double t = 1e30;
     if (allow_single) t = std::min(t, std::ceil(t1 * s / sms) / s);
-    if (allow_pair) t = std::min(t, std::ceil(t2 * s / pairs) / s / 1.03);
+    if (allow_pair) t = std::min(t, std::ceil(t2 * s / pairs) / s / 1.07);
     t += 0.023 * (s - 1) * (t1 / sms);
     if (t < best_t - 1e-9) {
       best_t = t;
