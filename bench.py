@@ -9,6 +9,7 @@ accumulation. Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
                   [--workload prefill|decode|int8|skewed] [--T ..] [--d ..] [--f ..]
+                  [--path auto|token_tile|weight_stream|token_tile_single] [--row-gather]
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica on its own GPU (the layer does not shard on this path): no data-path

@@ -1,6 +1,6 @@
 // gemm_common.cuh — pieces shared by the single-CTA and the CTA-pair grouped
 // expert GEMM kernels: tile constants, parameters, the device-side tile
-// scheduler data, the gate activation, the exact int8 -> bf16 conversion and the token-tile
+// scheduler data, the gate activation, the exact int8 -> fp16 conversion and the token-tile
 // epilogue (act(gate) * up -> bf16 H, or gate * down -> fp32 Y).
 #pragma once
 

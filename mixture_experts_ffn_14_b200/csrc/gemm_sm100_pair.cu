@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
       }
     }
   } else if (W8 && warp >= 8) {
-    // ----------------------------------------------- int8 -> bf16 convert --
+    // ----------------------------------------------- int8 -> fp16 convert --
     const int ct = threadIdx.x - 256;
     int stage = 0;
     uint32_t phase = 0;
