@@ -52,11 +52,17 @@ constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
 // flight: STAGES slots of [X tile | int8 W staging] (32 KB) filled by TMA, and
 // CSTAGES slots of converted fp16 W tiles (32 KB) that the converter warps fill
 // up to two stages ahead of the MMA (4 + 3 measured ~3 % faster than 5 + 2).
-template <bool W8>
+// TALL (int8 weights, token tiles): one tile covers 256 token rows; each
+// converted W tile serves two M = 128 MMAs (rows 0-127 into accumulator
+// columns 0-255, rows 128-255 into 256-511), so the conversion and the converted
+// tile's shared-memory traffic per FLOP halve. The two halves of TMEM then hold
+// one tile, and the epilogue no longer overlaps the next tile's main loop.
+template <bool W8, bool TALL = false>
 struct Cfg {
-  static constexpr int STAGES = 4;
-  static constexpr int SLOT_BYTES = X_BYTES + (W8 ? W8_BYTES : W_BYTES);
-  static constexpr int CSTAGES = W8 ? 3 : 0;
+  static constexpr int XS_BYTES = (TALL ? 2 : 1) * X_BYTES;
+  static constexpr int STAGES = TALL ? 3 : 4;
+  static constexpr int SLOT_BYTES = XS_BYTES + (W8 ? W8_BYTES : W_BYTES);
+  static constexpr int CSTAGES = W8 ? (TALL ? 2 : 3) : 0;
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
@@ -65,15 +71,21 @@ struct Cfg {
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
 constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ring
-static_assert(Cfg<true>::CSTAGES <= kMaxCStages, "converted-W ring deeper than its barrier slots");
+static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages,
+              "converted-W ring deeper than its barrier slots");
 static_assert((2 * Cfg<true>::STAGES + 2 * kMaxCStages + 4) * 8 + 16 + sizeof(SharedSched) <= Cfg<true>::BAR_BYTES,
               "barrier area too small");
+static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cfg<false>::SMEM <= 232448,
+              "shared memory above the per-block limit");
 
 template <int KIND, bool WS, bool W8>
 __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     moe_expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                            const __grid_constant__ CUtensorMap tm_w1, const Params p) {
-  using C = Cfg<W8>;
+  constexpr bool TALL = W8 && !WS;
+  constexpr int TROWS = TALL ? 2 * BM : BM;  // token rows per tile
+  constexpr int NACC = TALL ? 1 : 2;         // accumulator buffers in flight
+  using C = Cfg<W8, TALL>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-B swizzle atoms.
@@ -110,7 +122,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       mbar_init(&tempty_bar[b], 128);
     }
     *abort_flag = 0;
-    build_sched(*sched, p, BM);
+    build_sched(*sched, p, TROWS);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -146,11 +158,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
         int32_t rtok[4] = {0, 0, 0, 0};
         if (G) gather_rows(p, t, t.row0 + 4 * lane, rtok);
         const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
-        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : X_BYTES;
+        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : C::XS_BYTES;
         const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
         for (int kb = 0; kb < p.kb_per_split; ++kb) {
           int ok = 1;
@@ -164,7 +176,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             return;
           }
           uint8_t* xs = smem + stage * C::SLOT_BYTES;
-          uint8_t* ws = xs + X_BYTES;  // bf16 W tile, or the int8 staging (W8)
+          uint8_t* ws = xs + C::XS_BYTES;  // bf16 W tile, or the int8 staging (W8)
           uint8_t* w8 = ws;
           const int k0 = (t.kb0 + kb) * BK;
           if (!G || lane == 0) {
@@ -174,6 +186,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
                 tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
             } else if (!G) {
               tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
+              if (TALL) tma_load_2d(xs + X_BYTES, &tm_x, &full_bar[stage], k0, t.row0 + BM);
             }
             if (W8) {
               if (KIND == GATEUP) {
@@ -209,7 +222,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       }
     };
     if (!WS && KIND == GATEUP && p.row_token != nullptr) {
-      if constexpr (!WS && KIND == GATEUP) produce(std::true_type{});
+      if constexpr (!WS && KIND == GATEUP && !W8) produce(std::true_type{});
     } else if (lane == 0) {
       produce(std::false_type{});
     }
@@ -223,7 +236,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusMmaTimeout);
           *abort_flag = 1;
@@ -248,6 +261,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           tc_fence_after();
           const uint32_t xs = smem_u32(smem + stage * C::SLOT_BYTES);
           const uint32_t ws = W8 ? smem_u32(conv_area + cstage * W_BYTES) : xs + X_BYTES;
+          const bool second_half = TALL && t.rows > BM;  // rows 128..255 of a tall tile
 #pragma unroll
           for (int k16 = 0; k16 < BK / 16; ++k16) {
             const uint32_t accum = (kb | k16) != 0;
@@ -264,6 +278,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             } else {
               const uint64_t wdesc = smem_desc_sw128(ws + k16 * 2048, WCHUNK, 1024);
               umma_bf16(d_tmem, xdesc, wdesc, idesc, accum);
+              if (second_half)
+                umma_bf16(d_tmem + 256, smem_desc_sw128(xs + X_BYTES + k16 * 32, 16, 1024), wdesc, idesc, accum);
             }
           }
           umma_commit(&empty_bar[stage]);
@@ -280,7 +296,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           }
         }
         umma_commit(&tfull_bar[acc]);
-        if (++acc == 2) {
+        if (++acc == NACC) {
           acc = 0;
           acc_phase ^= 1;
         }
@@ -293,7 +309,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
       if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
@@ -302,7 +318,9 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * 256;
       if (!WS) {
-        epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, t.rows);
+        epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, min(t.rows, BM));
+        if (TALL && t.rows > BM)  // rows 128..255 of a tall tile: accumulator columns 256..511
+          epilogue_token_rows<KIND, W8>(p, t, tbase + 256, 32 * q + lane, t.row0 + BM, t.rows - BM);
       } else {
         // Weight-stream: TMEM lane = output column, TMEM column = token.
         const int ntok = ((t.rows + 15) / 16) * 16;
@@ -354,7 +372,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
-      if (++acc == 2) {
+      if (++acc == NACC) {
         acc = 0;
         acc_phase ^= 1;
       }
@@ -370,7 +388,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     int cstage = 0;
     uint32_t cphase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, BM, t); tile += gridDim.x) {
+    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
         if (!warp_wait(&full_bar[stage], phase, abort_flag) || !warp_wait(&cempty_bar[cstage], cphase ^ 1, abort_flag)) {
           atomicOr(p.status, kStatusConvertTimeout);
@@ -378,7 +396,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           goto convert_done;
         }
         {
-          const uint8_t* w8 = smem + stage * C::SLOT_BYTES + X_BYTES;
+          const uint8_t* w8 = smem + stage * C::SLOT_BYTES + C::XS_BYTES;
           uint8_t* wc = conv_area + cstage * W_BYTES;
 #pragma unroll
           for (int it = 0; it < 1024 / C::CONVERT_THREADS; ++it)
@@ -413,7 +431,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
 
 template <int KIND, bool WS, bool W8>
 cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
-  using C = Cfg<W8>;
+  constexpr bool TALL = W8 && !WS;
+  using C = Cfg<W8, TALL>;
   auto kern = moe_expert_gemm_kernel<KIND, WS, W8>;
   const cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
@@ -464,7 +483,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.status = a.status;
 
   // Upper bound of the tile count (the exact count is only known on device).
-  const int64_t mtiles_max = a.rows / BM + kE;
+  const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : BM) + kE;
   const int64_t tiles_max = mtiles_max * (a.N / p.ntile) * p.splits;
   const int grid = static_cast<int>(std::min<int64_t>(tiles_max, device_sm_count()));
   kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_x, tm_w0, tm_w1, p);

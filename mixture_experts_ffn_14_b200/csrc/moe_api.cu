@@ -173,13 +173,13 @@ bool use_weight_stream(int64_t T, moe_path_t path) {
 // 2.3 % of the unsplit work per extra split for the fp32 partial sums that are
 // written and read again (their bytes relative to the GEMM time at d, f).
 int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested, bool allow_single,
-                                      bool allow_pair) {
+                                      bool allow_pair, int64_t single_rows) {
   const int64_t kblocks = f / 64;
   if (requested > 0) return kblocks % requested == 0 ? requested : -1;
   auto valid = [&](int64_t s) { return s >= 1 && kblocks % s == 0 && kblocks / s >= 8; };
   const double per_expert = static_cast<double>(2 * T) / kE;
   const double nt = static_cast<double>(d / 256);
-  const double t1 = kE * (per_expert / 128.0 + 0.5) * nt;  // expected single-CTA tiles
+  const double t1 = kE * (per_expert / single_rows + 0.5) * nt;  // expected single-CTA tiles
   const double t2 = kE * (per_expert / 256.0 + 0.5) * nt;  // expected pair tiles
   const double sms = device_sm_count(), pairs = sms / 2;
   int32_t best = 1;
@@ -228,7 +228,9 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
     // Which token-tile forms may run (see the launch logic in run_forward).
     const bool allow_pair = path == MOE_PATH_TOKEN_TILE || (path == MOE_PATH_AUTO && dtype != MOE_BF16_INT8W);
     const bool allow_single = path != MOE_PATH_TOKEN_TILE;
-    L.splits = choose_token_tile_down_splits(T, d, f, down_splits, allow_single, allow_pair);
+    // int8 weights take 256-row single-CTA tiles (two MMAs per converted tile).
+    L.splits = choose_token_tile_down_splits(T, d, f, down_splits, allow_single, allow_pair,
+                                             dtype == MOE_BF16_INT8W ? 256 : 128);
   }
   // A requested split factor must divide the K blocks whichever path runs.
   if (down_splits > 0 && choose_down_splits(T, d, f, down_splits) < 1) L.splits = -1;
