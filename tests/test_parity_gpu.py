@@ -346,6 +346,19 @@ def test_int8_tile_boundaries(T):
         full_check(inp, gpu)
 
 
+@pytest.mark.parametrize("T,skew", [(516, False), (1028, False), (700, True)])
+def test_int8_tall_tiles_both_halves(T, skew):
+    # int8 token tiles hold 256 rows as two MMAs on one converted weight tile;
+    # the second (rows 128..255) runs only when the tile has more than 128 rows.
+    # About 130 and 257 rows per expert, and a skewed load (one expert near half
+    # of all slots), put tiles on both sides of 128 and 256.
+    inp = small_bf16(T, seed=95 + T, int8=True, skew=skew)
+    g = run_gpu(inp)
+    counts = g["counts"]
+    assert (counts % 256 > 128).any() or (counts > 256).any()
+    full_check(inp, g)
+
+
 @pytest.mark.parametrize("splits", [2, 3])
 def test_int8_token_tile_split_k(splits):
     inp = small_bf16(600, d=512, f=384, seed=91, int8=True)
