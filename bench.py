@@ -614,7 +614,9 @@ def run_decode(a, moe, W, wl, inp, dev, pk):
     # The same step captured once in a CUDA graph and replayed (no per-launch
     # host work, no stage events): what a serving loop that replays graphs sees.
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    # thread_local: CUDA calls of other threads (NCCL's, under torchrun) do not
+    # disturb the capture.
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
         run(xd, outd)
     torch.cuda.synchronize()
     for _ in range(a.warmup):
