@@ -197,14 +197,18 @@ MOE_EXPORT moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options
  * scratch fits. Returns MOE_ERR_WORKSPACE when the problem needs more than the
  * 32 MiB maximum (e.g. T = 64 at d = 6144, f = 32768 fits; T = 4096 does not).
  * The first call on a device looks up the array's device address and should
- * come before any stream capture. All calls on a device share the array:
- * calls that may overlap on the GPU race and must be ordered by the caller. */
+ * come before any stream capture; a call with T == 0 does only that set-up and
+ * launches nothing. All calls on a device share the array: calls that may
+ * overlap on the GPU race and must be ordered by the caller. The kernels'
+ * status word lives in the array; moe_device_status(NULL, ...) reads it. */
 MOE_EXPORT moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_options_t* opts,
                                             moe_stream_t stream);
 
 /* Synchronises `stream` and reads the status word that the kernels of the last
- * call on `workspace` recorded (NULL = the moe_forward cache of the current
- * device). Returns MOE_OK, MOE_ERR_DEVICE_CHECK (and the raw code in *code if
+ * call on `workspace` recorded. With workspace == NULL it reads the two
+ * library-owned words of the current device, the moe_forward cache's and the
+ * moe_forward_noalloc scratch's (each if it exists), and reports their OR.
+ * Returns MOE_OK, MOE_ERR_DEVICE_CHECK (and the raw code in *code if
  * code != NULL) or MOE_ERR_CUDA. */
 MOE_EXPORT moe_status_t moe_device_status(const void* workspace, moe_stream_t stream, uint32_t* code);
 

@@ -419,6 +419,10 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   return MOE_OK;
 }
 
+// Device address of the moe_forward_noalloc scratch's status word on device
+// `dev`, or nullptr while no noalloc call has set it up there.
+const void* noalloc_status_word(int dev);
+
 }  // namespace
 
 extern "C" {
@@ -477,23 +481,28 @@ moe_status_t moe_forward(const void* x, const float* w_router, const void* w_gat
 }
 
 moe_status_t moe_device_status(const void* workspace, moe_stream_t stream, uint32_t* code) {
-  const void* ws = workspace;
-  if (!ws) {
+  // The status words to read: the given workspace's, or with NULL both
+  // library-owned ones of the current device (the moe_forward cache and the
+  // moe_forward_noalloc scratch), whichever exist.
+  const void* words[2] = {workspace, nullptr};
+  if (!workspace) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_cache_mu);
-    if (static_cast<int>(g_cache.size()) <= dev || !g_cache[dev].ws) {
-      if (code) *code = 0;
-      return MOE_OK;
+    {
+      std::lock_guard<std::mutex> lk(g_cache_mu);
+      words[0] = static_cast<int>(g_cache.size()) > dev ? g_cache[dev].ws : nullptr;
     }
-    ws = g_cache[dev].ws;
+    words[1] = noalloc_status_word(dev);
   }
-  uint32_t v = 0;
+  uint32_t v[2] = {0, 0};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int i = 0; i < 2; ++i)
+    if (words[i] && cudaMemcpyAsync(&v[i], words[i], sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (code) *code = v;
-  return v == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
+  const uint32_t all = v[0] | v[1];
+  if (code) *code = all;
+  return all == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
 }
 
 const char* moe_status_string(moe_status_t s) {
@@ -545,6 +554,12 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 std::mutex g_noalloc_mu;
 std::vector<void*> g_noalloc_ptr;  // per device: device address of g_noalloc_scratch
 
+const void* noalloc_status_word(int dev) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  // run_forward keeps the status word at offset 0 of the scratch.
+  return static_cast<int>(g_noalloc_ptr.size()) > dev ? g_noalloc_ptr[dev] : nullptr;
+}
+
 // Device address of the scratch array on the current device (set up once).
 cudaError_t noalloc_scratch_address(void** out) {
   int dev = 0;
@@ -567,7 +582,12 @@ cudaError_t noalloc_scratch_address(void** out) {
 extern "C" moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_options_t* opts,
                                             moe_stream_t stream) {
   const moe_status_t st = check_args(args);
-  if (st != MOE_OK || args->T == 0) return st;
+  if (st != MOE_OK) return st;
+  // Look the scratch up first, so that a T == 0 call (which launches nothing)
+  // serves as the device's set-up call before any stream capture.
+  void* ws = nullptr;
+  if (noalloc_scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
+  if (args->T == 0) return MOE_OK;
   moe_options_t o{};
   if (opts) o = *opts;
   if (o.down_splits < 0) return MOE_ERR_INVALID_ARG;
@@ -586,7 +606,5 @@ extern "C" moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_op
     }
   }
   if (L.total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;  // problem too large for the fixed scratch
-  void* ws = nullptr;
-  if (noalloc_scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
   return run_forward(args, &o, nullptr, ws, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }

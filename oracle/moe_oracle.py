@@ -33,7 +33,7 @@ Sources (page title, section):
               item 3: the published code evaluates all 8 experts densely and keeps
               2 with a one-hot mask.
 
-Readings where the pages are silent, ambiguous or disagree (each also in the design doc):
+Readings where the pages are silent, ambiguous or disagree:
   R1  GELU is the tanh approximation 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))
       by default; [ch10] §10.4 writes GELU as z * Phi(z) (erf form), kept as mode "erf".
   R2  GELU is applied to the w_gate projection; w_up is linear; w_down projects back.
