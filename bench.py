@@ -338,13 +338,16 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 
 
 def launches_per_step(wl, path):
-    """Kernels of ours per step: router, dispatch, two GEMMs, combine; with the
-    automatic token-tile choice on bf16 weights each GEMM launches both forms
-    (the one not chosen returns at once); above 1024 router blocks (T > 32768)
-    a histogram scan runs before the dispatch."""
+    """Kernels of ours per step: router, dispatch, two GEMMs, and a combine
+    kernel on the weight-stream path (token tiles combine in the down
+    projection's epilogue); with the automatic token-tile choice on bf16
+    weights each GEMM launches both forms (the one not chosen returns at once);
+    above 1024 router blocks (T > 32768) a histogram scan runs before the
+    dispatch."""
+    ws = path == "weight_stream" or (path == "auto" and wl.T <= 256)
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
-    return 5 + (2 if both else 0) + (1 if scan else 0)
+    return 4 + (1 if ws else 0) + (2 if both else 0) + (1 if scan else 0)
 
 
 # ---------------------------------------------------------------- main --

@@ -147,6 +147,9 @@ typedef struct {
                                   on B200, where four-row gathers cannot feed the MMA).
                                   The weight-stream form always reads the copy;
                                   MOE_BF16_INT8W returns MOE_ERR_UNSUPPORTED with 1.      */
+  int32_t separate_combine;    /* 0: token tiles sum each token's two expert rows in the
+                                  down projection's epilogue (default); 1: a separate
+                                  combine kernel does it (same result bit for bit)       */
 } moe_options_t;
 
 /* Optional outputs for inspection; each is a device pointer or NULL.
@@ -163,7 +166,10 @@ typedef struct {
                           write the intermediate here                         */
 } moe_debug_t;
 
-/* Forward pass with a library-owned workspace: one cache per device, grown
+/* Passage: grok-field-guide "Grok-1 blueprint", section "MoE sublayer" (router,
+ * top-2, gated experts, gate-weighted sum); gates as in Grok-1 book ch. 10,
+ * section 10.3.1 (not renormalised); experts as in section 10.4 (GeGLU).
+ * Forward pass with a library-owned workspace: one cache per device, grown
  * with cudaMalloc when a call needs more (never shrunk), guarded by a mutex.
  * Calls on one device share that workspace, so calls that may overlap on the
  * GPU (different streams) must use moe_forward_ex with their own workspaces.
@@ -174,12 +180,24 @@ MOE_EXPORT moe_status_t moe_forward(const void* x, const float* w_router, const 
                          int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
                          moe_dtype_t dtype, moe_stream_t stream);
 
-/* Bytes of device workspace moe_forward_ex needs for these sizes (0 on bad
- * arguments). `path` and `down_splits` as in moe_options_t (0 = auto). */
+/* Passage: Grok-1 book ch. 11, section 11.3.1 item 3 (the sparse reorder and
+ * grouped GEMM that replace the dense one-hot evaluation need the permuted
+ * rows and intermediates this workspace holds).
+ * Bytes of device workspace moe_forward_ex needs for these sizes with the
+ * automatic kernel choices (path MOE_PATH_AUTO, automatic split-K), 0 on bad
+ * arguments or T == 0. 256-byte multiple. Host only: no CUDA call. */
 MOE_EXPORT size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
-                          moe_dtype_t dtype, moe_path_t path, int32_t down_splits);
+                                     moe_dtype_t dtype);
 
-/* Forward pass on a caller-provided device workspace of ws_bytes bytes
+/* The same for a call whose moe_options_t sets `path` and `down_splits`
+ * (0 = automatic), which change the workspace layout: 0 also when the split
+ * factor does not divide f / 64 or the path is unknown. */
+MOE_EXPORT size_t moe_workspace_size_ex(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
+                                        moe_dtype_t dtype, moe_path_t path, int32_t down_splits);
+
+/* Passage: as moe_forward; the options follow Grok-1 book ch. 10, section
+ * 10.3.1 (Mixtral renormalisation, sandwich post-norm) and section 10.4 (SiLU).
+ * Forward pass on a caller-provided device workspace of ws_bytes bytes
  * (256-byte aligned, at least moe_workspace_size(...)); allocates nothing.
  * `opts` and `dbg` may be NULL. Concurrent calls need distinct workspaces. */
 MOE_EXPORT moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options_t* opts,
@@ -204,7 +222,8 @@ MOE_EXPORT moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options
 MOE_EXPORT moe_status_t moe_forward_noalloc(const moe_args_t* args, const moe_options_t* opts,
                                             moe_stream_t stream);
 
-/* Synchronises `stream` and reads the status word that the kernels of the last
+/* No counterpart on the pages: the library's own failure reporting.
+ * Synchronises `stream` and reads the status word that the kernels of the last
  * call on `workspace` recorded. With workspace == NULL it reads the two
  * library-owned words of the current device, the moe_forward cache's and the
  * moe_forward_noalloc scratch's (each if it exists), and reports their OR.
@@ -224,10 +243,10 @@ MOE_EXPORT moe_status_t moe_device_status(const void* workspace, moe_stream_t st
  * arguments, MOE_ERR_CUDA if the launch fails. */
 MOE_EXPORT moe_status_t moe_selftest_bounded_wait(void* workspace, uint32_t limit_us, moe_stream_t stream);
 
-/* Static description of a status code (never NULL). */
+/* No counterpart on the pages. Static description of a status code (never NULL). */
 MOE_EXPORT const char* moe_status_string(moe_status_t status);
 
-/* Library ABI version, currently 1. */
+/* No counterpart on the pages. Library ABI version, currently 2. */
 MOE_EXPORT int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

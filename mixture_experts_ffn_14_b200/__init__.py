@@ -19,6 +19,7 @@ from ._native import (  # noqa: F401
 )
 
 __all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_forward_noalloc", "moe_workspace_size",
+           "moe_workspace_size_ex",
            "moe_device_status", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
            "dtype_code"]
 
@@ -77,7 +78,15 @@ def moe_abi_version() -> int:
 
 
 def moe_workspace_size(T, d, f, E=8, k=2, dtype=MOE_BF16, path=MOE_PATH_AUTO, down_splits=0) -> int:
-    return N.lib().moe_workspace_size(T, d, f, E, k, dtype, path, down_splits)
+    """Workspace bytes of a moe_forward_ex call; the C call with the automatic
+    kernel choices, or its _ex form when ``path`` / ``down_splits`` are set."""
+    if path == MOE_PATH_AUTO and down_splits == 0:
+        return N.lib().moe_workspace_size(T, d, f, E, k, dtype)
+    return N.lib().moe_workspace_size_ex(T, d, f, E, k, dtype, path, down_splits)
+
+
+def moe_workspace_size_ex(T, d, f, E=8, k=2, dtype=MOE_BF16, path=MOE_PATH_AUTO, down_splits=0) -> int:
+    return N.lib().moe_workspace_size_ex(T, d, f, E, k, dtype, path, down_splits)
 
 
 def moe_forward(x, w_router, w_gate, w_up, w_down, out, scales=None, stream=None):
@@ -94,7 +103,7 @@ def moe_forward(x, w_router, w_gate, w_up, w_down, out, scales=None, stream=None
 
 
 def _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual, post_norm_weight,
-             norm_eps, row_gather=False):
+             norm_eps, row_gather=False, separate_combine=False):
     ev = None
     if stage_events is not None:
         handles = [e.cuda_event for e in stage_events]
@@ -104,14 +113,14 @@ def _options(activation, router_bias, path, down_splits, stage_events, renormali
     opts = N.MoeOptions(activation, _ptr(router_bias), path, down_splits,
                         ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)) if ev is not None else None,
                         int(bool(renormalize)), _ptr(residual), _ptr(post_norm_weight), float(norm_eps),
-                        int(bool(row_gather)))
+                        int(bool(row_gather)), int(bool(separate_combine)))
     return opts, ev
 
 
 def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=None, router_bias=None,
                    activation=MOE_ACT_GELU_TANH, path=MOE_PATH_AUTO, down_splits=0, debug=None, stream=None,
                    stage_events=None, renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5,
-                   row_gather=False, raise_on_error=True):
+                   row_gather=False, separate_combine=False, raise_on_error=True):
     """Forward pass on a caller workspace (a uint8 CUDA tensor). ``debug`` is a
     dict with any of idx, gates, counts, offsets, perm_token, perm_slot, h.
     ``stage_events``: 6 torch.cuda.Event (already created, e.g. recorded once)
@@ -119,7 +128,9 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
     ``activation``, ``residual``, ``post_norm_weight`` / ``norm_eps``: the
     moe_options_t variants (Mixtral routing, SiLU, post-RMSNorm + residual).
     ``row_gather``: token tiles gather their gate/up rows from x with TMA row
-    gathers instead of reading the dispatch stage's permuted copy."""
+    gathers instead of reading the dispatch stage's permuted copy.
+    ``separate_combine``: sum each token's two expert rows in a combine kernel
+    instead of the down projection's epilogue (same result)."""
     T, d = x.shape
     E, _, f = w_gate.shape
     sc = _scales(scales)
@@ -127,7 +138,7 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
                      ctypes.pointer(sc) if sc is not None else None, _ptr(out), T, d, f, E, 2,
                      dtype_code(x, w_gate))
     opts, _keep = _options(activation, router_bias, path, down_splits, stage_events, renormalize, residual,
-                           post_norm_weight, norm_eps, row_gather)
+                           post_norm_weight, norm_eps, row_gather, separate_combine)
     dbg = None
     if debug:
         dbg = N.MoeDebug(*[_ptr(debug.get(n)) for n in

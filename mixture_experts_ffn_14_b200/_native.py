@@ -37,7 +37,8 @@ class MoeArgs(ctypes.Structure):
 class MoeOptions(ctypes.Structure):
     _fields_ = [("activation", c_int), ("router_bias", c_void_p), ("path", c_int), ("down_splits", c_int32),
                 ("stage_events", POINTER(c_void_p)), ("renormalize", c_int32), ("residual", c_void_p),
-                ("post_norm_weight", c_void_p), ("norm_eps", c_float), ("row_gather", c_int32)]
+                ("post_norm_weight", c_void_p), ("norm_eps", c_float), ("row_gather", c_int32),
+                ("separate_combine", c_int32)]
 
 
 class MoeDebug(ctypes.Structure):
@@ -48,7 +49,8 @@ class MoeDebug(ctypes.Structure):
 EXPORTS.update({
     "moe_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(MoeScales), c_void_p,
                             c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_void_p]),
-    "moe_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_int, c_int32]),
+    "moe_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int32, c_int]),
+    "moe_workspace_size_ex": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_int, c_int32]),
     "moe_forward_ex": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), POINTER(MoeDebug), c_void_p, c_size_t,
                                c_void_p]),
     "moe_forward_noalloc": (c_int, [POINTER(MoeArgs), POINTER(MoeOptions), c_void_p]),

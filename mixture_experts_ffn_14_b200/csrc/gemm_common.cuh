@@ -46,6 +46,12 @@ struct Params {
   int32_t sm_count;      // SMs of the device (same value for both token-tile kernels)
   int32_t* tile_counter; // CTA-pair kernel, bf16 weights: tiles handed out in order (zero on entry)
   uint32_t* status;
+  // DOWN token tiles with the combine in the epilogue (combine_count != nullptr)
+  const int32_t* perm_token;
+  const int32_t* slot_pos;
+  int32_t* combine_count;
+  __nv_bfloat16* combine_out;
+  const __nv_bfloat16* residual;
 };
 
 enum { kRunAlways = 0, kRunIfPair = 1, kRunIfSingle = 2 };
@@ -233,10 +239,83 @@ __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t*
   convert_store_segment(src, wtile, sp);
 }
 
+// ---- combine in the down-projection epilogue ----------------------------
+// Token t's output row is the sum of 2 * splits gate-scaled fp32 pieces: one
+// per (slot, K split), each produced by a different tile (the two slots are
+// different experts). Every piece is stored in Y[split, permuted row] by the
+// epilogue that produced it, which then counts itself on the arrival counter
+// of (t, column tile) after a fence. The epilogue whose arrival completes the
+// count (it never waits: everything it needs is already in memory) sums the
+// pieces in a fixed order, slot 0 over splits, then slot 1 over splits, then
+// the two, adds the residual row if any, and stores the bf16 output: the result
+// does not depend on which tile finished last, and no output is updated with
+// atomics.
+
+// Fixed-order sum of the 2 * splits pieces of token `tok`, columns n0 + 8 * lane
+// .. + 7, read from L2 (other SMs wrote them), stored as bf16.
+__device__ __forceinline__ void combine_columns(const Params& p, int tok, int n0, int lane) {
+  const int64_t p0 = p.slot_pos[2 * static_cast<int64_t>(tok)];
+  const int64_t p1 = p.slot_pos[2 * static_cast<int64_t>(tok) + 1];
+  const int64_t c = n0 + 8 * lane;
+  const float* y = static_cast<const float*>(p.out);
+  float a[8], b[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = b[j] = 0.0f;
+  for (int s = 0; s < p.splits; ++s) {
+    const float4* r0 = reinterpret_cast<const float4*>(y + s * p.split_stride + p0 * p.N + c);
+    const float4* r1 = reinterpret_cast<const float4*>(y + s * p.split_stride + p1 * p.N + c);
+    const float4 u0 = __ldcg(r0), u1 = __ldcg(r0 + 1), v0 = __ldcg(r1), v1 = __ldcg(r1 + 1);
+    a[0] += u0.x; a[1] += u0.y; a[2] += u0.z; a[3] += u0.w;
+    a[4] += u1.x; a[5] += u1.y; a[6] += u1.z; a[7] += u1.w;
+    b[0] += v0.x; b[1] += v0.y; b[2] += v0.z; b[3] += v0.w;
+    b[4] += v1.x; b[5] += v1.y; b[6] += v1.z; b[7] += v1.w;
+  }
+  float o[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = a[j] + b[j];
+  const int64_t at = static_cast<int64_t>(tok) * p.N + c;
+  if (p.residual != nullptr) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p.residual + at);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o[2 * j] += __uint_as_float(w[j] << 16);
+      o[2 * j + 1] += __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+  *reinterpret_cast<uint4*>(p.combine_out + at) =
+      make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+}
+
+// Called by a whole epilogue warp after each lane stored its row's piece of
+// this tile (valid rows only). Lanes whose arrival completes a token's count
+// hand the token to the warp, which combines one token row per pass with
+// coalesced 1 KB reads.
+__device__ __forceinline__ void combine_arrive(const Params& p, const Tile& t, int64_t row, bool valid) {
+  int tok = 0;
+  bool last = false;
+  if (valid) {
+    tok = p.perm_token[row];
+    __threadfence();  // this lane's piece is visible device-wide before it is counted
+    const int old = atomicAdd(&p.combine_count[static_cast<int64_t>(tok) * (p.N / 256) + t.n0 / 256], 1);
+    last = old == 2 * p.splits - 1;
+  }
+  unsigned m = __ballot_sync(0xffffffffu, last);
+  if (m == 0) return;
+  __threadfence();  // the counted pieces of other SMs are read after the count
+  const int lane = threadIdx.x % 32;
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    combine_columns(p, __shfl_sync(0xffffffffu, tok, src), t.n0, lane);
+  }
+}
+
 // Token-tile epilogue of one epilogue warp: TMEM lane = token row r (0..127 of
 // this CTA's rows starting at permuted row `row_base`), 256 accumulator
 // columns. GATEUP: columns 0..127 gate, 128..255 up -> H[row, n0 + c] (bf16; fp16 with int8 weights).
-// DOWN: 256 output columns -> fp32 Y[split, row, n0 + c] = acc * gate[row].
+// DOWN: 256 output columns -> fp32 Y[split, row, n0 + c] = acc * gate[row],
+// then (combine_count set) the combine above.
 template <int KIND, bool W8>
 __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile& t, uint32_t tbase, int r,
                                                     int64_t row_base, int nvalid) {
@@ -291,6 +370,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
         for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
       }
     }
+    if (p.combine_count != nullptr) combine_arrive(p, t, row, valid);
   }
 }
 

@@ -481,6 +481,12 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.select = a.select;
   p.sm_count = device_sm_count();
   p.status = a.status;
+  const bool fuse = KIND == DOWN && !WS && a.combine_count != nullptr;
+  p.perm_token = fuse ? a.perm_token : nullptr;
+  p.slot_pos = fuse ? a.slot_pos : nullptr;
+  p.combine_count = fuse ? a.combine_count : nullptr;
+  p.combine_out = fuse ? static_cast<__nv_bfloat16*>(a.combine_out) : nullptr;
+  p.residual = fuse ? static_cast<const __nv_bfloat16*>(a.residual) : nullptr;
 
   // Upper bound of the tile count (the exact count is only known on device).
   const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : BM) + kE;

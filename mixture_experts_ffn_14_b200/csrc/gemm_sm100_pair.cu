@@ -491,6 +491,12 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   p.select = a.select;
   p.sm_count = device_sm_count();
   p.status = a.status;
+  const bool fuse = KIND == DOWN && a.combine_count != nullptr;
+  p.perm_token = fuse ? a.perm_token : nullptr;
+  p.slot_pos = fuse ? a.slot_pos : nullptr;
+  p.combine_count = fuse ? a.combine_count : nullptr;
+  p.combine_out = fuse ? static_cast<__nv_bfloat16*>(a.combine_out) : nullptr;
+  p.residual = fuse ? static_cast<const __nv_bfloat16*>(a.residual) : nullptr;
 
   const int64_t ptiles_max = (a.rows / PAIR_ROWS + kE) * (a.N / p.ntile) * p.splits;
   const int pairs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ptiles_max, max_pairs)));

@@ -1,7 +1,8 @@
 // moe_api.cu — the C ABI (include/moe.h): argument checks, workspace planning,
 // TMA descriptor encoding and the launch sequence
-//   router -> dispatch -> expert gate/up GEMM -> expert down GEMM -> combine
-// on the caller's stream, with no host synchronisation.
+//   router -> dispatch -> expert gate/up GEMM -> expert down GEMM (+ combine)
+// on the caller's stream, with no host synchronisation. Token tiles combine in
+// the down projection's epilogue; the other paths run a combine kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -243,6 +244,9 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   L.router_slices = router_slices(T, d, dtype);
   L.status = take(kAlign);
   L.arrivals = take(sizeof(int32_t) * L.nblk);  // right after the status word: one memset clears both
+  // Token tiles: arrival counters of the combine in the down-projection
+  // epilogue, one per (token, 256-column tile); cleared by the same memset.
+  L.combine_count = L.tile_path ? take(sizeof(int32_t) * T * (d / 256)) : o;
   L.idx = take(sizeof(int32_t) * rows);
   L.gates = take(sizeof(float) * rows);
   L.hist = take(sizeof(int32_t) * L.nblk * kE);
@@ -279,6 +283,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE) return MOE_ERR_INVALID_ARG;
   if (o->down_splits < 0) return MOE_ERR_INVALID_ARG;
   if (o->row_gather != 0 && o->row_gather != 1) return MOE_ERR_INVALID_ARG;
+  if (o->separate_combine != 0 && o->separate_combine != 1) return MOE_ERR_INVALID_ARG;
   // The int8-weight GEMMs take fp16 activations from the dispatch copy; a row
   // gather would feed them x's bf16 rows.
   if (o->row_gather == 1 && a->dtype == MOE_BF16_INT8W) return MOE_ERR_UNSUPPORTED;
@@ -314,6 +319,11 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   void* h = h_ext ? dbg->h : static_cast<void*>(ws + L.h);
   float* y = reinterpret_cast<float*>(ws + L.y);
   const int64_t T = a->T, d = a->d, f = a->f;
+  // Token tiles sum each token's two rows in the down projection's epilogue;
+  // a separate combine kernel runs for the weight-stream and fp32 paths, with
+  // the post-RMSNorm (it needs whole rows), or when asked for.
+  const bool fused_combine = L.tile_path && !o->post_norm_weight && o->separate_combine == 0;
+  int32_t* combine_count = reinterpret_cast<int32_t*>(ws + L.combine_count);
 
 #define MOE_TRY(call)                                  \
   do {                                                 \
@@ -323,8 +333,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   auto mark = [&](int i) {
     return o->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(o->stage_events[i]), stream) : cudaSuccess;
   };
-  // Status word and router arrival counters start at zero.
-  MOE_TRY(cudaMemsetAsync(status, 0, L.arrivals + sizeof(int32_t) * L.nblk - L.status, stream));
+  // Status word, router arrival counters and combine arrival counters start at
+  // zero (contiguous regions, up to the next one).
+  MOE_TRY(cudaMemsetAsync(status, 0, L.idx - L.status, stream));
   MOE_TRY(mark(0));
   MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, L.router_slices,
                         logits_part, arrivals, idx, gates, hist, stream));
@@ -397,11 +408,19 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g2.N = static_cast<int32_t>(d);
     g2.splits = L.splits;
     g2.tile_counter = tile_counters + 1;
+    if (fused_combine) {
+      g2.perm_token = perm_token;
+      g2.slot_pos = slot_pos;
+      g2.combine_count = combine_count;
+      g2.combine_out = a->out;
+      g2.residual = o->residual;
+    }
     MOE_TRY(launch_gemm(g2, true));
   }
   MOE_TRY(mark(4));
-  MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, o->residual, o->post_norm_weight,
-                         o->norm_eps, a->out, stream));
+  if (!fused_combine)
+    MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, o->residual, o->post_norm_weight,
+                           o->norm_eps, a->out, stream));
   MOE_TRY(mark(5));
 
   if (dbg) {
@@ -434,8 +453,8 @@ moe_status_t moe_forward_ex(const moe_args_t* args, const moe_options_t* opts, c
   return run_forward(args, opts, dbg, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
-size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k, moe_dtype_t dtype,
-                          moe_path_t path, int32_t down_splits) {
+size_t moe_workspace_size_ex(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k, moe_dtype_t dtype,
+                             moe_path_t path, int32_t down_splits) {
   moe_args_t a{};
   a.T = T;
   a.d = d;
@@ -451,13 +470,17 @@ size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
   return L.total;
 }
 
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k, moe_dtype_t dtype) {
+  return moe_workspace_size_ex(T, d, f, E, k, dtype, MOE_PATH_AUTO, 0);
+}
+
 moe_status_t moe_forward(const void* x, const float* w_router, const void* w_gate, const void* w_up,
                          const void* w_down, const moe_scales_t* w_scales, void* out, int64_t T, int64_t d,
                          int64_t f, int32_t E, int32_t k, moe_dtype_t dtype, moe_stream_t stream) {
   moe_args_t a{x, w_router, w_gate, w_up, w_down, w_scales, out, T, d, f, E, k, dtype};
   const moe_status_t st = check_args(&a);
   if (st != MOE_OK || T == 0) return st;
-  const size_t need = moe_workspace_size(T, d, f, E, k, dtype, MOE_PATH_AUTO, 0);
+  const size_t need = moe_workspace_size(T, d, f, E, k, dtype);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_cache_mu);
@@ -518,7 +541,7 @@ const char* moe_status_string(moe_status_t s) {
   return "unknown status";
 }
 
-int32_t moe_abi_version(void) { return 1; }
+int32_t moe_abi_version(void) { return 2; }
 
 }  // extern "C"
 

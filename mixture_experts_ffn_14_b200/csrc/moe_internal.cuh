@@ -28,7 +28,7 @@ enum : uint32_t {
 
 // Byte offsets of the regions of one call's workspace (each 256-aligned).
 struct WorkspaceLayout {
-  size_t status, arrivals, idx, gates, hist, hist_pre, logits_part, counts, offsets, perm_token, perm_slot,
+  size_t status, arrivals, combine_count, idx, gates, hist, hist_pre, logits_part, counts, offsets, perm_token, perm_slot,
       slot_pos, gate_perm;
   size_t xp, h, y, total;
   int64_t nblk;      // router / dispatch CTAs
@@ -100,6 +100,14 @@ struct TcGemmArgs {
   int32_t select;           // 0: always run; 1 / 2: run only if the pair / single token-tile form is preferred
   int32_t* tile_counter;    // pair form: zeroed int that hands out tiles in order, or nullptr (static order)
   uint32_t* status;
+  // DOWN token tiles: the combine in the epilogue (out[t] = sum of the two
+  // gate-scaled rows of token t, in fixed order). combine_count == nullptr:
+  // the epilogue only writes Y and a separate combine kernel runs.
+  const int32_t* perm_token;  // [rows] token of each permuted row
+  const int32_t* slot_pos;    // [T, 2] permuted row of each (token, slot)
+  int32_t* combine_count;     // [T, N/256] arrivals per (token, column tile), zero on entry
+  void* combine_out;          // [T, N] bf16 sublayer output
+  const void* residual;       // [T, N] bf16 added to the output, or nullptr
 };
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);

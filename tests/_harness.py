@@ -24,7 +24,7 @@ def np64(t) -> np.ndarray:
 
 def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, activation=moe.MOE_ACT_GELU_TANH, down_splits=0, want_h=True,
             stream=None, renormalize=False, residual=None, post_norm_weight=None, norm_eps=1e-5,
-            row_gather=False) -> dict:
+            row_gather=False, separate_combine=False) -> dict:
     """One forward through moe_forward_ex with every debug output requested."""
     x = inp["x"]
     T, d = x.shape
@@ -48,7 +48,7 @@ def run_gpu(inp: dict, *, path=moe.MOE_PATH_AUTO, activation=moe.MOE_ACT_GELU_TA
     moe.moe_forward_ex(x, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws, scales=scales,
                        router_bias=inp.get("router_bias"), activation=activation, path=path, down_splits=down_splits,
                        renormalize=renormalize, residual=residual, post_norm_weight=post_norm_weight,
-                       norm_eps=norm_eps, row_gather=row_gather,
+                       norm_eps=norm_eps, row_gather=row_gather, separate_combine=separate_combine,
                        debug=dbg, stream=stream)
     torch.cuda.synchronize()
     st, code = moe.moe_device_status(ws)

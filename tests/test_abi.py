@@ -36,7 +36,7 @@ def test_every_declared_function_is_exported():
 
 
 def test_status_strings_and_version():
-    assert moe.moe_abi_version() == 1
+    assert moe.moe_abi_version() == 2
     texts = {moe.moe_status_string(s) for s in range(7)}
     assert len(texts) == 7
     assert moe.moe_status_string(99) == "unknown status"
@@ -62,6 +62,9 @@ def test_workspace_size_rules():
     eight = ws(64, 6144, 32768, path=moe.MOE_PATH_WEIGHT_STREAM, down_splits=8)
     assert eight - one >= 7 * 128 * 6144 * 4
     assert ws(64, 6144, 32768) % 256 == 0
+    # the six-argument C call is the _ex call with the automatic choices
+    for T, d, f, dt in ((4096, 6144, 32768, 1), (64, 6144, 32768, 1), (1024, 6144, 32768, 2), (64, 128, 256, 0)):
+        assert N.lib().moe_workspace_size(T, d, f, 8, 2, dt) == N.lib().moe_workspace_size_ex(T, d, f, 8, 2, dt, 0, 0)
 
 
 def _args(T=64, d=512, f=384, E=8, k=2, dtype=moe.MOE_BF16, base=0x10000000):

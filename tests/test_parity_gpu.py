@@ -256,6 +256,33 @@ def test_bitwise_determinism_and_streams():
     assert np.array_equal(a["perm_token"], b["perm_token"])
 
 
+@pytest.mark.parametrize("T,path,int8,splits,residual,skew", [
+    (300, moe.MOE_PATH_TOKEN_TILE, False, 1, False, False),
+    (300, moe.MOE_PATH_TOKEN_TILE_SINGLE, False, 3, True, False),
+    (1000, moe.MOE_PATH_AUTO, False, 0, False, False),
+    (700, moe.MOE_PATH_AUTO, False, 2, True, True),
+    (600, moe.MOE_PATH_AUTO, True, 2, True, False),
+    (517, moe.MOE_PATH_TOKEN_TILE_SINGLE, True, 1, False, True),
+])
+def test_fused_combine_matches_combine_kernel_bitwise(T, path, int8, splits, residual, skew):
+    # Token tiles sum each token's rows in the down projection's epilogue
+    # (whichever tile finishes last, in a fixed order); the separate combine
+    # kernel sums the same pieces in the same order: outputs equal bit for bit,
+    # also with split-K pieces, the residual add, int8 tiles and skewed loads.
+    inp = small_bf16(T, seed=110 + T, int8=int8, skew=skew)
+    kw = {}
+    if residual:
+        g = torch.Generator(device=DEV)
+        g.manual_seed(T)
+        kw["residual"] = torch.randn(inp["x"].shape, generator=g, device=DEV).to(torch.bfloat16)
+    a = run_gpu(inp, path=path, down_splits=splits, want_h=False, **kw)
+    b = run_gpu(inp, path=path, down_splits=splits, want_h=False, separate_combine=True, **kw)
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["out"], b["out"])
+    okw = {"residual": kw["residual"]} if residual else {}
+    full_check(inp, a, check_h=False, **okw)
+
+
 def test_moe_forward_library_workspace_matches_ex():
     inp = small_bf16(257, seed=32)
     out = torch.empty_like(inp["x"])
