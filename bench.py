@@ -51,6 +51,8 @@ def parse():
                     help="kernel family (default: the library's automatic choice)")
     ap.add_argument("--row-gather", action="store_true",
                     help="token tiles gather their gate/up rows from x (TMA row gather) instead of the copy")
+    ap.add_argument("--separate-combine", action="store_true",
+                    help="sum each token's rows in the combine kernel instead of the down projection's epilogue")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode (T=64) side measurement")
     ap.add_argument("--no-int8", action="store_true", help="skip the int8-weight (T=1024) side measurement")
     ap.add_argument("--no-skewed", action="store_true", help="skip the skewed-load (T=16384) side measurement")
@@ -276,11 +278,12 @@ class Runner:
 
     PATHS = {"auto": 0, "token_tile": 1, "weight_stream": 2, "token_tile_single": 3}
 
-    def __init__(self, moe, inp, T, d, f, dev, path="auto", row_gather=False):
+    def __init__(self, moe, inp, T, d, f, dev, path="auto", row_gather=False, separate_combine=False):
         import torch
 
         self.moe, self.inp = moe, inp
         self.row_gather = row_gather
+        self.separate_combine = separate_combine
         self.path = self.PATHS[path]
         dt = moe.dtype_code(inp["x"], inp["w_gate"])
         self.ws = torch.empty(moe.moe_workspace_size(T, d, f, dtype=dt, path=self.path), dtype=torch.uint8,
@@ -291,7 +294,8 @@ class Runner:
         i = self.inp
         self.moe.moe_forward_ex(x, i["w_router"], i["w_gate"], i["w_up"], i["w_down"], out, self.ws,
                                 scales=self.scales, router_bias=i.get("router_bias"), stage_events=events,
-                                debug=debug, path=self.path, row_gather=self.row_gather)
+                                debug=debug, path=self.path, row_gather=self.row_gather,
+                                separate_combine=self.separate_combine)
 
 
 def timed_steps(run, x, out, K, flush, clk=None):
@@ -384,7 +388,7 @@ def main():
 
     T, d, f = wl.T, wl.d, wl.f
     inp = W.make_torch(wl, dev)
-    run = Runner(moe, inp, T, d, f, dev, a.path, a.row_gather)
+    run = Runner(moe, inp, T, d, f, dev, a.path, a.row_gather, a.separate_combine)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     counts = torch.empty(8, dtype=torch.int32, device=dev)
@@ -464,10 +468,11 @@ def main():
         "expert_slots": expert_counts,
         "path": a.path,
         "row_gather": bool(a.row_gather),
+        "combine": "combine kernel" if a.separate_combine else "in the down projection's epilogue (token tiles)",
         "hbm_gbs_weights": round(world * K * wbytes / (t_max / 1e3) / 1e9, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,
-        "gpu_launches": launches_per_step(wl, a.path) * K,
+        "gpu_launches": (launches_per_step(wl, a.path) + (1 if a.separate_combine and wl.T > 256 else 0)) * K,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                    "power_w_max": clocks.get("power_w_max"), "power_w_median": clocks.get("power_w_median"),
                    "samples": clocks.get("samples"), "source": clocks.get("source")},

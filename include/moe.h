@@ -40,10 +40,19 @@
  * Errors. Arguments are checked on the host before anything is launched; a
  * failed check returns its status and launches nothing. A launch failure
  * returns MOE_ERR_CUDA. Faults of earlier asynchronous work surface at the
- * caller's next synchronisation, not here. Kernels never trap: a wait that
- * exceeds its time limit records a code in the workspace status word, which
- * moe_device_status() reads back as MOE_ERR_DEVICE_CHECK. Behaviour on
- * non-finite inputs is unspecified.
+ * caller's next synchronisation, not here. Kernels never trap: they record
+ * what went wrong as bits of the workspace status word, which
+ * moe_device_status() reads back as MOE_ERR_DEVICE_CHECK with the code:
+ *   0x01, 0x02, 0x04, 0x08  a GEMM wait (producer, MMA, epilogue, int8
+ *                           converter) exceeded its time limit; the kernel
+ *                           unwound and the output is incomplete
+ *   0x10                    moe_selftest_bounded_wait's wait ran out (expected)
+ *   0x20                    MOE_BF16_INT8W: an activation or GeGLU intermediate
+ *                           left the fp16 range (|v| > 65504 became infinite);
+ *                           the output is not valid
+ *   0x40                    library built with MOE_DEBUG_BOUNDS: an index
+ *                           outside its array was caught and the access skipped
+ * Behaviour on non-finite inputs is unspecified.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H
@@ -195,6 +204,99 @@ MOE_EXPORT size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int32_t E,
 MOE_EXPORT size_t moe_workspace_size_ex(int64_t T, int64_t d, int64_t f, int32_t E, int32_t k,
                                         moe_dtype_t dtype, moe_path_t path, int32_t down_splits);
 
+/* ---- Expert parallelism ----------------------------------------------------
+ * Passage: Grok-1 book ch. 1, section 1.6.3 (the MoE layer shards the expert
+ * axis over the devices of a (1, 8) mesh with shard_map). Building blocks of
+ * that form on W GPUs, one process each, GPU r owning n = 8 / W consecutive
+ * experts: each GPU routes and dispatches its own tokens (moe_route_dispatch;
+ * the permuted rows are then grouped by owning GPU, because the permutation is
+ * expert-major), the caller's communication library sends every block of rows
+ * to its owner, the owner makes the received rows expert-contiguous
+ * (moe_gather_rows), runs its experts on them (moe_experts_forward, which
+ * also applies each row's gate), the rows go back the same way, and each GPU
+ * sums its tokens' two rows (moe_combine). With the same split-K factor the
+ * result equals moe_forward_ex's bit for bit. Every pointer is a device
+ * pointer; workspaces are 256-byte aligned device memory of at least the
+ * stated size; each call records its status word at the start of its
+ * workspace (moe_device_status reads it). */
+
+/* Outputs of moe_route_dispatch (device arrays owned by the caller). */
+typedef struct {
+  int32_t* idx;        /* [T, 2] chosen experts, slot 0 = larger logit          */
+  float* gates;        /* [T, 2] their gates                                     */
+  int32_t* counts;     /* [8]    token slots per expert                          */
+  int32_t* offsets;    /* [9]    exclusive prefix of counts                      */
+  int32_t* perm_token; /* [2T]   token of each permuted row                      */
+  int32_t* perm_slot;  /* [2T]   slot of each permuted row                       */
+  int32_t* slot_pos;   /* [T, 2] permuted row of each (token, slot)              */
+  float* gate_perm;    /* [2T]   gate of each permuted row                       */
+  void* xp;            /* [2T, d] x rows in permuted order: x's dtype, but fp16
+                          for MOE_BF16_INT8W (the int8-weight GEMMs' operand)    */
+} moe_routed_t;
+
+/* Workspace bytes of moe_route_dispatch (0 on bad sizes or T == 0). */
+MOE_EXPORT size_t moe_route_workspace_size(int64_t T, int64_t d, moe_dtype_t dtype);
+
+/* The router and dispatch stages of moe_forward on T tokens: logits, softmax,
+ * top-2 (gates renormalised if renormalize == 1), counts, offsets, the stable
+ * (expert, token) permutation and the permuted copy of x. Same size limits
+ * and errors as moe_forward_ex. */
+MOE_EXPORT moe_status_t moe_route_dispatch(const void* x, const float* w_router, const float* router_bias,
+                                           int64_t T, int64_t d, moe_dtype_t dtype, int32_t renormalize,
+                                           const moe_routed_t* routed, void* workspace, size_t ws_bytes,
+                                           moe_stream_t stream);
+
+/* Rows for n_experts experts held by this GPU (row block e belongs to local
+ * expert e, in order). */
+typedef struct {
+  const void* xp;              /* [R, d] rows, expert-contiguous: bf16 (MOE_BF16), fp16
+                                  (MOE_BF16_INT8W) or fp32 (MOE_F32)                  */
+  const int32_t* counts;       /* [n_experts] rows of each local expert (device)      */
+  const float* gate;           /* [R] gate of each row, or NULL for 1                 */
+  const void* w_gate;          /* [n_experts, d, f]                                   */
+  const void* w_up;            /* [n_experts, d, f]                                   */
+  const void* w_down;          /* [n_experts, f, d]                                   */
+  const moe_scales_t* w_scales;/* MOE_BF16_INT8W: [n_experts, f], [n_experts, f],
+                                  [n_experts, d]; else NULL                           */
+  float* y;                    /* [R, d] fp32: gate * FFN_e(row)                       */
+  int64_t R, d, f;
+  int32_t n_experts;           /* 1 .. 8 */
+  moe_dtype_t dtype;
+} moe_expert_rows_t;
+
+/* Workspace bytes of moe_experts_forward (0 on bad sizes, R == 0 or a split
+ * factor that does not divide f / 64). `path` and `down_splits` as in
+ * moe_options_t. */
+MOE_EXPORT size_t moe_experts_workspace_size(int64_t R, int64_t d, int64_t f, int32_t n_experts,
+                                             moe_dtype_t dtype, moe_path_t path, int32_t down_splits);
+
+/* The expert GEMMs of moe_forward on rows already grouped by expert:
+ * y[r] = gate[r] * down(act(xp[r] . w_gate[e]) * (xp[r] . w_up[e])) for the
+ * rows r of local expert e (section 10.4 of ch. 10; activation, path and
+ * down_splits from opts, NULL = defaults). Token-tile rows run on single CTAs
+ * unless opts->path is MOE_PATH_TOKEN_TILE (CTA pairs). */
+MOE_EXPORT moe_status_t moe_experts_forward(const moe_expert_rows_t* rows, const moe_options_t* opts,
+                                            void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* out[t] = y[slot_pos[t,0]] + y[slot_pos[t,1]] (fp32 sum, in that order, then
+ * cast to the x dtype: fp32 for MOE_F32, else bf16), with the post-RMSNorm
+ * and residual add of moe_options_t when post_norm_weight / residual are set
+ * (the blueprint's gate-weighted sum; ch. 10, section 10.3.1 sandwich norm).
+ * y is [2T, d] fp32 in permuted order. Workspace: at least 256 bytes. */
+MOE_EXPORT moe_status_t moe_combine(const float* y, const int32_t* slot_pos, int64_t T, int64_t d,
+                                    moe_dtype_t dtype, const void* residual, const float* post_norm_weight,
+                                    float norm_eps, void* out, void* workspace, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* No counterpart on the pages (data movement of the expert-parallel form):
+ * dst row i = src row index[i] (int32, device), for i < n; rows of row_bytes
+ * bytes, a multiple of 4 (src and dst 4-byte aligned) or of 16 (16-byte
+ * aligned, copied in 16-byte vectors); src has src_rows rows. Workspace: at
+ * least 256 bytes. */
+MOE_EXPORT moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* index, int64_t n,
+                                        int64_t row_bytes, void* dst, void* workspace, size_t ws_bytes,
+                                        moe_stream_t stream);
+
 /* Passage: as moe_forward; the options follow Grok-1 book ch. 10, section
  * 10.3.1 (Mixtral renormalisation, sandwich post-norm) and section 10.4 (SiLU).
  * Forward pass on a caller-provided device workspace of ws_bytes bytes
@@ -248,6 +350,13 @@ MOE_EXPORT const char* moe_status_string(moe_status_t status);
 
 /* No counterpart on the pages. Library ABI version, currently 2. */
 MOE_EXPORT int32_t moe_abi_version(void);
+
+/* No counterpart on the pages. Options the library was compiled with, as bits:
+ * MOE_BUILD_DEBUG_BOUNDS = the MOE_DEBUG_BOUNDS build (every index that one
+ * kernel computes and another uses is checked before the access; a failed
+ * check sets status bit 0x40 and skips the access; slower, for testing). */
+#define MOE_BUILD_DEBUG_BOUNDS 1
+MOE_EXPORT int32_t moe_build_flags(void);
 
 #ifdef __cplusplus
 }

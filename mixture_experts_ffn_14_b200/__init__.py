@@ -19,7 +19,7 @@ from ._native import (  # noqa: F401
 )
 
 __all__ = ["MoeError", "moe_forward", "moe_forward_ex", "moe_forward_noalloc", "moe_workspace_size",
-           "moe_workspace_size_ex",
+           "moe_workspace_size_ex", "moe_build_flags",
            "moe_device_status", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
            "dtype_code"]
 
@@ -75,6 +75,11 @@ def moe_status_string(status: int) -> str:
 
 def moe_abi_version() -> int:
     return N.lib().moe_abi_version()
+
+
+def moe_build_flags() -> int:
+    """Build options of the loaded library (bit MOE_BUILD_DEBUG_BOUNDS)."""
+    return N.lib().moe_build_flags()
 
 
 def moe_workspace_size(T, d, f, E=8, k=2, dtype=MOE_BF16, path=MOE_PATH_AUTO, down_splits=0) -> int:

@@ -11,7 +11,13 @@ import ctypes
 import os
 from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+# The library to load: the normal build, or another build of the same sources
+# (e.g. libmoe_b200_debug.so, the MOE_DEBUG_BOUNDS build) named by
+# MOE_B200_LIBRARY (a file name inside the package, or a path).
+LIB_NAME = os.environ.get("MOE_B200_LIBRARY", "libmoe_b200.so")
+LIB_PATH = LIB_NAME if os.path.isabs(LIB_NAME) else os.path.join(PKG_DIR, LIB_NAME)
+MOE_BUILD_DEBUG_BOUNDS = 1
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 3
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK = 4, 5, 6
@@ -46,6 +52,18 @@ class MoeDebug(ctypes.Structure):
                 ("perm_token", c_void_p), ("perm_slot", c_void_p), ("h", c_void_p)]
 
 
+class MoeRouted(ctypes.Structure):
+    _fields_ = [("idx", c_void_p), ("gates", c_void_p), ("counts", c_void_p), ("offsets", c_void_p),
+                ("perm_token", c_void_p), ("perm_slot", c_void_p), ("slot_pos", c_void_p),
+                ("gate_perm", c_void_p), ("xp", c_void_p)]
+
+
+class MoeExpertRows(ctypes.Structure):
+    _fields_ = [("xp", c_void_p), ("counts", c_void_p), ("gate", c_void_p), ("w_gate", c_void_p),
+                ("w_up", c_void_p), ("w_down", c_void_p), ("w_scales", POINTER(MoeScales)), ("y", c_void_p),
+                ("R", c_int64), ("d", c_int64), ("f", c_int64), ("n_experts", c_int32), ("dtype", c_int)]
+
+
 EXPORTS.update({
     "moe_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(MoeScales), c_void_p,
                             c_int64, c_int64, c_int64, c_int32, c_int32, c_int, c_void_p]),
@@ -58,6 +76,16 @@ EXPORTS.update({
     "moe_selftest_bounded_wait": (c_int, [c_void_p, c_uint32, c_void_p]),
     "moe_status_string": (c_char_p, [c_int]),
     "moe_abi_version": (c_int32, []),
+    "moe_build_flags": (c_int32, []),
+    "moe_route_workspace_size": (c_size_t, [c_int64, c_int64, c_int]),
+    "moe_route_dispatch": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int, c_int32,
+                                   POINTER(MoeRouted), c_void_p, c_size_t, c_void_p]),
+    "moe_experts_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32, c_int, c_int, c_int32]),
+    "moe_experts_forward": (c_int, [POINTER(MoeExpertRows), POINTER(MoeOptions), c_void_p, c_size_t, c_void_p]),
+    "moe_combine": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p, c_float, c_void_p,
+                            c_void_p, c_size_t, c_void_p]),
+    "moe_gather_rows": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_size_t,
+                                c_void_p]),
 })
 
 _LIB = None

@@ -1,8 +1,14 @@
 """Build the CUDA library ``libmoe_b200.so`` in-tree with nvcc for sm_100a.
 
-Usage: ``python -m mixture_experts_ffn_14_b200.build [--force] [--verbose]``.
+Usage: ``python -m mixture_experts_ffn_14_b200.build [--force] [--verbose] [--debug-bounds]``.
 Objects go to ``mixture_experts_ffn_14_b200/_build/`` and are rebuilt when a
 source or header is newer than the object. Cross-compiles without a GPU.
+
+``--debug-bounds`` builds ``libmoe_b200_debug.so`` from the same sources with
+``-DMOE_DEBUG_BOUNDS`` (objects in ``_build_debug/``): every index one kernel
+computes and another uses is checked before the access, a failed check sets
+status bit 0x40 and skips the access. Load it with
+``MOE_B200_LIBRARY=libmoe_b200_debug.so``.
 """
 
 from __future__ import annotations
@@ -19,6 +25,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libmoe_b200_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [
@@ -45,25 +53,27 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug_bounds: bool = False) -> str:
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug_bounds else (BUILD, LIB)
+    flags = NVCC_FLAGS + (["-DMOE_DEBUG_BOUNDS"] if debug_bounds else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     objs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or ptxas_info or _stale(obj, [src] + hdrs):
-            cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", src, "-o", obj]
+            cmd = [nvcc()] + flags + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", src, "-o", obj]
             if verbose:
                 print(" ".join(cmd), flush=True)
             subprocess.run(cmd, check=True)
-    if force or _stale(LIB, objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart_static", "-ldl", "-lpthread", "-lrt"]
+    if force or _stale(lib, objs):
+        cmd = [nvcc()] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart_static", "-ldl", "-lpthread", "-lrt"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-    return LIB
+    return lib
 
 
 def main(argv=None):
@@ -71,8 +81,10 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers / spills per kernel")
+    ap.add_argument("--debug-bounds", action="store_true",
+                    help="build libmoe_b200_debug.so with the device-side index checks")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info))
+    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info, debug_bounds=a.debug_bounds))
 
 
 if __name__ == "__main__":

@@ -120,6 +120,10 @@ __device__ __forceinline__ void build_sched(SharedSched& s, const Params& p, int
     acc += s.mt[e] * nt_count * p.splits;
   }
   s.pre[kE] = acc;
+  if (kDebugBounds && !expert_blocks_ok(p.counts, p.offsets, kE, p.rows)) {
+    atomicOr(p.status, kStatusBounds);
+    s.pre[kE] = 0;  // no tile: every role sees the same empty schedule
+  }
 }
 
 __device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& p, int tile, int tile_rows,
@@ -138,6 +142,10 @@ __device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& 
   t.rows = min(tile_rows, s.cnt[e] - mt * tile_rows);
   t.n0 = nt * p.ntile;
   t.kb0 = ks * p.kb_per_split;
+  if (kDebugBounds && !tile_ok(t.row0, t.rows, p.rows, t.n0, p.ntile, p.N)) {
+    atomicOr(p.status, kStatusBounds);
+    return false;  // every role decodes the same tile and stops here
+  }
   return true;
 }
 
@@ -162,6 +170,11 @@ __device__ __forceinline__ float act_f32(float z, int mode) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Nonzero if either fp16 half of `h` is infinite or NaN (exponent all ones).
+__device__ __forceinline__ uint32_t f16x2_nonfinite(uint32_t h) {
+  return static_cast<uint32_t>((h & 0x7C00u) == 0x7C00u) | static_cast<uint32_t>((h & 0x7C000000u) == 0x7C000000u);
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -256,6 +269,10 @@ __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t*
 __device__ __forceinline__ void combine_columns(const Params& p, int tok, int n0, int lane) {
   const int64_t p0 = p.slot_pos[2 * static_cast<int64_t>(tok)];
   const int64_t p1 = p.slot_pos[2 * static_cast<int64_t>(tok) + 1];
+  if (kDebugBounds && !(index_ok(p0, p.rows) && index_ok(p1, p.rows))) {
+    if (lane == 0) atomicOr(p.status, kStatusBounds);
+    return;
+  }
   const int64_t c = n0 + 8 * lane;
   const float* y = static_cast<const float*>(p.out);
   float a[8], b[8];
@@ -296,6 +313,13 @@ __device__ __forceinline__ void combine_arrive(const Params& p, const Tile& t, i
   bool last = false;
   if (valid) {
     tok = p.perm_token[row];
+    if (kDebugBounds && !index_ok(tok, p.rows / 2)) {
+      atomicOr(p.status, kStatusBounds);
+      valid = false;
+      tok = 0;
+    }
+  }
+  if (valid) {
     __threadfence();  // this lane's piece is visible device-wide before it is counted
     const int old = atomicAdd(&p.combine_count[static_cast<int64_t>(tok) * (p.N / 256) + t.n0 / 256], 1);
     last = old == 2 * p.splits - 1;
@@ -323,6 +347,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
   const int64_t row = row_base + r;
   if (KIND == GATEUP) {
     uint16_t* hout = static_cast<uint16_t*>(p.out);
+    uint32_t f16_bad = 0;  // int8 weights: an H value beyond the fp16 range
 #pragma unroll 1
     for (int c = 0; c < 128; c += 32) {
       uint32_t g[32], u[32];
@@ -342,6 +367,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
         // int8 weights run the MMAs on fp16 operands, so H is stored as fp16 there.
         const float h0 = act_f32(g0, p.act) * u0, h1 = act_f32(g1, p.act) * u1;
         packed[j / 2] = W8 ? pack_f16x2(h0, h1) : pack_bf16x2(h0, h1);
+        if (W8) f16_bad |= f16x2_nonfinite(packed[j / 2]);
       }
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);
@@ -350,6 +376,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
           dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       }
     }
+    if (W8 && valid && f16_bad) atomicOr(p.status, kStatusFp16Range);
   } else {
     float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
     const float gate = valid ? p.gate_perm[row] : 0.0f;

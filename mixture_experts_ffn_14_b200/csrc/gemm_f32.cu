@@ -23,7 +23,8 @@ struct F32Sched {
   int cnt[kE], off[kE], mt[kE], pre[kE + 1];
 };
 
-__device__ __forceinline__ void load_sched(F32Sched& s, const int32_t* counts, const int32_t* offsets, int nt) {
+__device__ __forceinline__ void load_sched(F32Sched& s, const int32_t* counts, const int32_t* offsets, int nt,
+                                           int64_t rows_total, uint32_t* status) {
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int e = 0; e < kE; ++e) {
@@ -34,6 +35,10 @@ __device__ __forceinline__ void load_sched(F32Sched& s, const int32_t* counts, c
       acc += s.mt[e] * nt;
     }
     s.pre[kE] = acc;
+    if (kDebugBounds && !expert_blocks_ok(counts, offsets, kE, rows_total)) {
+      atomicOr(status, kStatusBounds);
+      s.pre[kE] = 0;  // no tile: nothing is read or written through these rows
+    }
   }
   __syncthreads();
 }
@@ -52,13 +57,14 @@ __global__ void __launch_bounds__(256) moe_f32_expert_gemm(const float* __restri
                                                            const int32_t* __restrict__ counts,
                                                            const int32_t* __restrict__ offsets,
                                                            const float* __restrict__ rowscale, int K, int N,
-                                                           int act, float* __restrict__ out) {
+                                                           int act, float* __restrict__ out, int64_t rows_total,
+                                                           uint32_t* __restrict__ status) {
   __shared__ F32Sched sched;
   __shared__ float As[TK][TM];
   __shared__ float Bs0[TK][TN];
   __shared__ float Bs1[DUAL ? TK : 1][DUAL ? TN : 1];
   const int nt = N / TN;
-  load_sched(sched, counts, offsets, nt);
+  load_sched(sched, counts, offsets, nt, rows_total, status);
   const int tid = threadIdx.x;
   const int ty = tid / 16, tx = tid % 16;
 
@@ -140,16 +146,19 @@ int f32_grid(int64_t T, int64_t N) {
 
 cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,
                               const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t act,
-                              float* h, cudaStream_t s) {
+                              float* h, uint32_t* status, cudaStream_t s) {
   moe_f32_expert_gemm<true><<<f32_grid(T, f), 256, 0, s>>>(xp, wg, wu, counts, offsets, nullptr,
-                                                          static_cast<int>(d), static_cast<int>(f), act, h);
+                                                          static_cast<int>(d), static_cast<int>(f), act, h, 2 * T,
+                                                          status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_f32_down(const float* h, const float* wd, const int32_t* counts, const int32_t* offsets,
-                            const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, cudaStream_t s) {
+                            const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, uint32_t* status,
+                            cudaStream_t s) {
   moe_f32_expert_gemm<false><<<f32_grid(T, d), 256, 0, s>>>(h, wd, nullptr, counts, offsets, gate_perm,
-                                                           static_cast<int>(f), static_cast<int>(d), 0, y);
+                                                           static_cast<int>(f), static_cast<int>(d), 0, y, 2 * T,
+                                                           status);
   return cudaGetLastError();
 }
 

@@ -332,6 +332,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             sg = __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + n]);
             su = __bfloat162float(p.s1[static_cast<int64_t>(t.e) * p.N + n]);
           }
+          uint32_t f16_bad = 0;  // int8 weights: an H value beyond the fp16 range
 #pragma unroll 1
           for (int c = 0; c < ntok; c += 32) {
             uint32_t g[32], u[32];
@@ -340,11 +341,14 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             for (int j = 0; j < 32; ++j) {
               if (c + j < t.rows) {
                 const float h = act_f32(__uint_as_float(g[j]) * sg, p.act) * (__uint_as_float(u[j]) * su);
-                hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] =
+                const uint16_t hv =
                     W8 ? __half_as_ushort(__float2half_rn(h)) : __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                if (W8) f16_bad |= static_cast<uint32_t>((hv & 0x7C00u) == 0x7C00u);
+                hout[static_cast<int64_t>(t.row0 + c + j) * p.N + n] = hv;
               }
             }
           }
+          if (W8 && f16_bad) atomicOr(p.status, kStatusFp16Range);
         } else {
           float* yout = static_cast<float*>(p.out) + static_cast<int64_t>(t.kb0 / p.kb_per_split) * p.split_stride;
           const int n_a = t.n0 + 32 * q + lane;
@@ -450,7 +454,8 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), kE};
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
+                              static_cast<uint64_t>(a.n_experts > 0 ? a.n_experts : kE)};
     const uint64_t esz = W8 ? 1 : 2;
     const uint64_t strides[2] = {static_cast<uint64_t>(a.N) * esz, static_cast<uint64_t>(a.N) * a.K * esz};
     const uint32_t box[3] = {static_cast<uint32_t>(W8 ? 128 : 64), BK, 1};

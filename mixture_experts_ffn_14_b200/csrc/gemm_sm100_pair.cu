@@ -460,7 +460,8 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), kE};
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
+                              static_cast<uint64_t>(a.n_experts > 0 ? a.n_experts : kE)};
     const uint64_t esz = W8 ? 1 : 2;
     const uint64_t strides[2] = {static_cast<uint64_t>(a.N) * esz, static_cast<uint64_t>(a.N) * a.K * esz};
     const uint32_t box[3] = {static_cast<uint32_t>(W8 ? 128 : 64), BK, 1};

@@ -341,15 +341,15 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
                         logits_part, arrivals, idx, gates, hist, stream));
   MOE_TRY(mark(1));
   MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, hist_pre, counts, offsets, perm_token,
-                          perm_slot, slot_pos, gate_perm, xp, stream));
+                          perm_slot, slot_pos, gate_perm, xp, status, stream));
   MOE_TRY(mark(2));
   if (a->dtype == MOE_F32) {
     MOE_TRY(launch_f32_gateup(static_cast<const float*>(xp), static_cast<const float*>(a->w_gate),
                               static_cast<const float*>(a->w_up), counts, offsets, T, d, f, o->activation,
-                              static_cast<float*>(h), stream));
+                              static_cast<float*>(h), status, stream));
     MOE_TRY(mark(3));
     MOE_TRY(launch_f32_down(static_cast<const float*>(h), static_cast<const float*>(a->w_down), counts, offsets,
-                            gate_perm, T, d, f, y, stream));
+                            gate_perm, T, d, f, y, status, stream));
   } else {
     const bool w8 = a->dtype == MOE_BF16_INT8W;
     TcGemmArgs g{};
@@ -420,7 +420,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   MOE_TRY(mark(4));
   if (!fused_combine)
     MOE_TRY(launch_combine(a->dtype, y, 2 * T * d, L.splits, slot_pos, T, d, o->residual, o->post_norm_weight,
-                           o->norm_eps, a->out, stream));
+                           o->norm_eps, a->out, status, stream));
   MOE_TRY(mark(5));
 
   if (dbg) {
@@ -542,6 +542,299 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 int32_t moe_abi_version(void) { return 2; }
+
+int32_t moe_build_flags(void) { return kDebugBounds ? MOE_BUILD_DEBUG_BOUNDS : 0; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Expert-parallel building blocks (Grok-1 book ch. 1, section 1.6.3: the MoE
+// layer shards the expert axis over the devices of the mesh). A forward over
+// W GPUs routes and dispatches each GPU's own tokens (moe_route_dispatch),
+// sends each block of rows to the GPU that owns its experts, runs the local
+// experts on the rows it received (moe_experts_forward, after moe_gather_rows
+// has made them expert-contiguous), sends the gate-scaled rows back and sums
+// each token's two rows (moe_combine). The exchanges themselves belong to the
+// caller's communication library.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct RouteLayout {
+  size_t status, arrivals, logits_part, hist, hist_pre, total;
+  int64_t nblk;
+  int32_t slices;
+};
+
+RouteLayout plan_route(int64_t T, int64_t d, moe_dtype_t dtype) {
+  RouteLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
+  L.slices = router_slices(T, d, dtype);
+  L.status = take(kAlign);
+  L.arrivals = take(sizeof(int32_t) * L.nblk);
+  L.logits_part = L.slices > 1 ? take(sizeof(float) * L.slices * T * kE) : 0;
+  L.hist = take(sizeof(int32_t) * L.nblk * kE);
+  L.hist_pre = take(sizeof(int32_t) * (L.nblk + 1) * kE);
+  L.total = o;
+  return L;
+}
+
+struct ExpertsLayout {
+  size_t status, counts, offsets, ones, h, ypart, total;
+  int32_t splits;
+  bool weight_stream;
+};
+
+bool experts_sizes_ok(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype_t dtype) {
+  moe_args_t a{};
+  a.T = (R + 1) / 2;
+  a.d = d;
+  a.f = f;
+  a.E = kE;
+  a.k = kK;
+  a.dtype = dtype;
+  return R >= 0 && R <= (int64_t(1) << 25) && n >= 1 && n <= kE && check_sizes(&a) == MOE_OK;
+}
+
+ExpertsLayout plan_experts(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype_t dtype, moe_path_t path,
+                           int32_t down_splits) {
+  ExpertsLayout L{};
+  // Weight-stream tiles when the local experts hold few rows on average
+  // (<= 64, as in the whole-layer choice), token tiles otherwise.
+  L.weight_stream = dtype != MOE_F32 && (path == MOE_PATH_WEIGHT_STREAM ||
+                                         (path == MOE_PATH_AUTO && R <= 64 * static_cast<int64_t>(n)));
+  const int64_t kblocks = f / 64;
+  if (down_splits > 0) {
+    L.splits = kblocks % down_splits == 0 && dtype != MOE_F32 ? down_splits : (down_splits == 1 ? 1 : -1);
+  } else if (L.weight_stream) {
+    // Enough tiles for ~10 waves, at least 8 K blocks per split.
+    const int64_t base = (R / 128 + n) * (d / 256);
+    int64_t best = 1;
+    for (int64_t s = 1; s <= 64; ++s) {
+      if (kblocks % s != 0 || kblocks / s < 8) continue;
+      best = s;
+      if (base * s >= 10 * static_cast<int64_t>(device_sm_count())) break;
+    }
+    L.splits = static_cast<int32_t>(best);
+  } else {
+    L.splits = 1;
+  }
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.counts = take(sizeof(int32_t) * kE);
+  L.offsets = take(sizeof(int32_t) * (kE + 1));
+  L.ones = take(sizeof(float) * std::max<int64_t>(R, 1));
+  L.h = take(act_bytes(dtype) * std::max<int64_t>(R, 1) * f);
+  L.ypart = L.splits > 1 ? take(sizeof(float) * L.splits * R * d) : o;
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_route_workspace_size(int64_t T, int64_t d, moe_dtype_t dtype) {
+  moe_args_t a{};
+  a.T = T;
+  a.d = d;
+  a.f = 128;
+  a.E = kE;
+  a.k = kK;
+  a.dtype = dtype;
+  if (T <= 0 || check_sizes(&a) != MOE_OK) return 0;
+  return plan_route(T, d, dtype).total;
+}
+
+moe_status_t moe_route_dispatch(const void* x, const float* w_router, const float* router_bias, int64_t T,
+                                int64_t d, moe_dtype_t dtype, int32_t renormalize, const moe_routed_t* r,
+                                void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  moe_args_t a{};
+  a.T = T;
+  a.d = d;
+  a.f = 128;
+  a.E = kE;
+  a.k = kK;
+  a.dtype = dtype;
+  moe_status_t st = check_sizes(&a);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !r || !r->idx || !r->gates || !r->counts || !r->offsets || !r->perm_token ||
+      !r->perm_slot || !r->slot_pos || !r->gate_perm || !r->xp)
+    return MOE_ERR_INVALID_ARG;
+  if (renormalize != 0 && renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(r->xp) || (router_bias && !aligned16(router_bias)))
+    return MOE_ERR_MISALIGNED;
+  const RouteLayout L = plan_route(T, d, dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < L.total)
+    return MOE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  if (cudaMemsetAsync(status, 0, L.logits_part ? L.logits_part - L.status : L.hist - L.status, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_router(dtype, x, w_router, router_bias, T, d, renormalize, L.slices,
+                    L.slices > 1 ? reinterpret_cast<float*>(ws + L.logits_part) : nullptr,
+                    reinterpret_cast<int32_t*>(ws + L.arrivals), r->idx, r->gates, hist, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_dispatch(dtype, x, T, d, L.nblk, r->idx, r->gates, hist, reinterpret_cast<int32_t*>(ws + L.hist_pre),
+                      r->counts, r->offsets, r->perm_token, r->perm_slot, r->slot_pos, r->gate_perm, r->xp, status,
+                      s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+size_t moe_experts_workspace_size(int64_t R, int64_t d, int64_t f, int32_t n_experts, moe_dtype_t dtype,
+                                  moe_path_t path, int32_t down_splits) {
+  if (R <= 0 || !experts_sizes_ok(R, d, f, n_experts, dtype)) return 0;
+  if (path < MOE_PATH_AUTO || path > MOE_PATH_TOKEN_TILE_SINGLE || down_splits < 0) return 0;
+  const ExpertsLayout L = plan_experts(R, d, f, n_experts, dtype, path, down_splits);
+  return L.splits < 1 ? 0 : L.total;
+}
+
+moe_status_t moe_experts_forward(const moe_expert_rows_t* a, const moe_options_t* opts, void* workspace,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  const moe_options_t defaults{};
+  const moe_options_t* o = opts ? opts : &defaults;
+  if (a->dtype != MOE_F32 && a->dtype != MOE_BF16 && a->dtype != MOE_BF16_INT8W) return MOE_ERR_INVALID_ARG;
+  if (a->R < 0 || a->d <= 0 || a->f <= 0 || a->n_experts < 1 || a->n_experts > kE) return MOE_ERR_INVALID_ARG;
+  if (!experts_sizes_ok(a->R, a->d, a->f, a->n_experts, a->dtype)) return MOE_ERR_UNSUPPORTED;
+  if (a->R == 0) return MOE_OK;
+  if (o->activation < MOE_ACT_GELU_TANH || o->activation > MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
+  if (o->path < MOE_PATH_AUTO || o->path > MOE_PATH_TOKEN_TILE_SINGLE || o->down_splits < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!a->xp || !a->counts || !a->w_gate || !a->w_up || !a->w_down || !a->y) return MOE_ERR_INVALID_ARG;
+  const bool w8 = a->dtype == MOE_BF16_INT8W;
+  if (w8 && (!a->w_scales || !a->w_scales->s_gate || !a->w_scales->s_up || !a->w_scales->s_down))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a->xp) || !aligned16(a->w_gate) || !aligned16(a->w_up) || !aligned16(a->w_down) ||
+      !aligned16(a->y))
+    return MOE_ERR_MISALIGNED;
+  if (w8 && (!aligned16(a->w_scales->s_gate) || !aligned16(a->w_scales->s_up) || !aligned16(a->w_scales->s_down)))
+    return MOE_ERR_MISALIGNED;
+  const ExpertsLayout L = plan_experts(a->R, a->d, a->f, a->n_experts, a->dtype, o->path, o->down_splits);
+  if (L.splits < 1) return MOE_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < L.total)
+    return MOE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  float* ones = reinterpret_cast<float*>(ws + L.ones);
+  void* h = ws + L.h;
+  const int64_t R = a->R, d = a->d, f = a->f;
+  const float* gate = a->gate ? a->gate : ones;
+  if (cudaMemsetAsync(status, 0, kAlign, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_local_schedule(a->counts, a->n_experts, counts, offsets, a->gate ? nullptr : ones, R, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // The row-count-based launch sizes of the kernels take T = R / 2 (R rows).
+  const int64_t T_eq = (R + 1) / 2;
+  if (a->dtype == MOE_F32) {
+    if (launch_f32_gateup(static_cast<const float*>(a->xp), static_cast<const float*>(a->w_gate),
+                          static_cast<const float*>(a->w_up), counts, offsets, T_eq, d, f, o->activation,
+                          static_cast<float*>(h), status, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_f32_down(static_cast<const float*>(h), static_cast<const float*>(a->w_down), counts, offsets, gate,
+                        T_eq, d, f, a->y, status, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  float* y = L.splits > 1 ? reinterpret_cast<float*>(ws + L.ypart) : a->y;
+  TcGemmArgs g{};
+  g.x = a->xp;
+  g.x_rows = R;
+  g.w0 = a->w_gate;
+  g.w1 = a->w_up;
+  g.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_gate) : nullptr;
+  g.s1 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_up) : nullptr;
+  g.counts = counts;
+  g.offsets = offsets;
+  g.gate_perm = gate;
+  g.out = h;
+  g.rows = R;
+  g.K = static_cast<int32_t>(d);
+  g.N = static_cast<int32_t>(f);
+  g.splits = 1;
+  g.act = o->activation;
+  g.int8_weights = w8;
+  g.weight_stream = L.weight_stream;
+  g.status = status;
+  g.n_experts = a->n_experts;
+  // One token-tile form per call here (the single-CTA one unless the pair form
+  // is asked for): the device-side choice between them needs zeroed tile
+  // counters that this workspace does not keep.
+  const bool pair = !L.weight_stream && o->path == MOE_PATH_TOKEN_TILE;
+  auto gemm = [&](const TcGemmArgs& args, bool down) -> cudaError_t {
+    if (pair) return down ? launch_tc_down_pair(args, s) : launch_tc_gateup_pair(args, s);
+    return down ? launch_tc_down(args, s) : launch_tc_gateup(args, s);
+  };
+  if (gemm(g, false) != cudaSuccess) return MOE_ERR_CUDA;
+  TcGemmArgs g2 = g;
+  g2.x = h;
+  g2.w0 = a->w_down;
+  g2.w1 = nullptr;
+  g2.s0 = w8 ? static_cast<const __nv_bfloat16*>(a->w_scales->s_down) : nullptr;
+  g2.s1 = nullptr;
+  g2.out = y;
+  g2.K = static_cast<int32_t>(f);
+  g2.N = static_cast<int32_t>(d);
+  g2.splits = L.splits;
+  if (gemm(g2, true) != cudaSuccess) return MOE_ERR_CUDA;
+  if (L.splits > 1 && launch_sum_splits(y, R * d, L.splits, R * d, a->y, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_combine(const float* y, const int32_t* slot_pos, int64_t T, int64_t d, moe_dtype_t dtype,
+                         const void* residual, const float* post_norm_weight, float norm_eps, void* out,
+                         void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || d % 4 != 0 || T > (int64_t(1) << 24)) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_F32 && dtype != MOE_BF16 && dtype != MOE_BF16_INT8W) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !slot_pos || !out) return MOE_ERR_INVALID_ARG;
+  if (post_norm_weight && !(norm_eps > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out) || (residual && !aligned16(residual)) ||
+      (post_norm_weight && !aligned16(post_norm_weight)))
+    return MOE_ERR_MISALIGNED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < kAlign)
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, kAlign, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_combine(dtype, y, 2 * T * d, 1, slot_pos, T, d, residual, post_norm_weight, norm_eps, out, status,
+                        s) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* index, int64_t n,
+                             int64_t row_bytes, void* dst, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (n < 0 || src_rows < 0 || row_bytes <= 0 || row_bytes % 4 != 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!src || !index || !dst) return MOE_ERR_INVALID_ARG;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst);
+  if ((a & (row_bytes % 16 == 0 ? 15u : 3u)) != 0) return MOE_ERR_MISALIGNED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < kAlign)
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, kAlign, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_gather_rows(src, src_rows, index, n, row_bytes, dst, status, s) == cudaSuccess ? MOE_OK
+                                                                                             : MOE_ERR_CUDA;
+}
 
 }  // extern "C"
 

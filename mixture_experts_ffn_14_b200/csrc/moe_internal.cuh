@@ -10,6 +10,7 @@
 #include <cstdint>
 
 #include "../../include/moe.h"
+#include "bounds.cuh"
 
 namespace moe {
 
@@ -24,6 +25,12 @@ enum : uint32_t {
   kStatusEpilogueTimeout = 1u << 2,
   kStatusConvertTimeout = 1u << 3,
   kStatusSelftestTimeout = 1u << 4,
+  // int8-weight path: an activation or GeGLU intermediate outside the fp16
+  // range (|v| > 65504 rounds to infinity) in the conversion to fp16.
+  kStatusFp16Range = 1u << 5,
+  // MOE_DEBUG_BOUNDS builds: an index outside its array was caught and the
+  // access skipped.
+  kStatusBounds = 1u << 6,
 };
 
 // Byte offsets of the regions of one call's workspace (each 256-aligned).
@@ -63,20 +70,31 @@ constexpr int64_t kDispatchSumBlocks = 1024;
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* hist_pre,
                             int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
-                            int32_t* slot_pos, float* gate_perm, void* xp,
+                            int32_t* slot_pos, float* gate_perm, void* xp, uint32_t* status,
                             cudaStream_t s);  // xp == nullptr: no row copy
 
 // out[t] = residual[t] + norm(y0 + y1); residual and norm_weight may be NULL.
+// Expert-parallel pieces: counts of n local experts -> the kE-slot counts and
+// offsets the GEMM kernels read (zero rows for the other slots), plus 1.0 gates
+// for rows without one; the fixed-order sum of split-K partials; a row gather.
+cudaError_t launch_local_schedule(const int32_t* counts_in, int32_t n, int32_t* counts, int32_t* offsets,
+                                  float* ones, int64_t n_ones, cudaStream_t s);
+cudaError_t launch_sum_splits(const float* part, int64_t split_stride, int32_t splits, int64_t n, float* y,
+                              cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, int64_t src_rows, const int32_t* index, int64_t n,
+                               int64_t row_bytes, void* dst, uint32_t* status, cudaStream_t s);
+
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
                            const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
-                           const float* norm_weight, float norm_eps, void* out, cudaStream_t s);
+                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s);
 
 // fp32 (SIMT) grouped expert GEMMs.
 cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,
                               const int32_t* offsets, int64_t T, int64_t d, int64_t f, int32_t act,
-                              float* h, cudaStream_t s);
+                              float* h, uint32_t* status, cudaStream_t s);
 cudaError_t launch_f32_down(const float* h, const float* wd, const int32_t* counts, const int32_t* offsets,
-                            const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, cudaStream_t s);
+                            const float* gate_perm, int64_t T, int64_t d, int64_t f, float* y, uint32_t* status,
+                            cudaStream_t s);
 
 // tcgen05 grouped expert GEMMs (bf16 or int8 weights).
 struct TcGemmArgs {
@@ -100,6 +118,7 @@ struct TcGemmArgs {
   int32_t select;           // 0: always run; 1 / 2: run only if the pair / single token-tile form is preferred
   int32_t* tile_counter;    // pair form: zeroed int that hands out tiles in order, or nullptr (static order)
   uint32_t* status;
+  int32_t n_experts;        // experts in the weight arrays (0 = kE); experts past it have no rows
   // DOWN token tiles: the combine in the epilogue (out[t] = sum of the two
   // gate-scaled rows of token t, in fixed order). combine_count == nullptr:
   // the epilogue only writes Y and a separate combine kernel runs.

@@ -292,6 +292,16 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
 }
+// Nonzero if one of the eight fp16 values is infinite or NaN (exponent field
+// all ones): a bf16 input of magnitude above 65504 overflowed in the conversion.
+__device__ __forceinline__ uint32_t f16x8_nonfinite(uint4 h) {
+  uint32_t bad = 0;
+  const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    bad |= static_cast<uint32_t>((w[i] & 0x7C00u) == 0x7C00u) | static_cast<uint32_t>((w[i] & 0x7C000000u) == 0x7C000000u);
+  return bad;
+}
 
 // Same 32-token range per CTA as the router. Each CTA sums the per-CTA
 // histograms to find where its tokens land (no cross-CTA waiting), ranks its
@@ -305,7 +315,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
     const float* __restrict__ gates, const int32_t* __restrict__ hist, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
     int32_t* __restrict__ slot_pos, float* __restrict__ gate_perm, TX* __restrict__ xp,
-    const int32_t* __restrict__ hist_pre, const int32_t* __restrict__ hist_tot) {
+    const int32_t* __restrict__ hist_pre, const int32_t* __restrict__ hist_tot, uint32_t* __restrict__ status) {
   // blockIdx.y splits the row gather of the block across gridDim.y CTAs; all of
   // them rank the block's tokens (cheap), the first one writes the permutation.
   __shared__ int red[8][2 * kE];
@@ -386,7 +396,13 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
       if (a == e) pa = r;
       if (b == e) pb = r;
     }
-    if (valid && blockIdx.y == 0) {
+    bool ok = valid;
+    if (kDebugBounds && valid && !(index_ok(pa, 2 * T) && index_ok(pb, 2 * T))) {
+      atomicOr(status, kStatusBounds);  // an expert id outside [0, E): skip the token
+      ok = false;
+      pa = pb = -1;
+    }
+    if (ok && blockIdx.y == 0) {
       perm_token[pa] = static_cast<int32_t>(t);
       perm_slot[pa] = 0;
       perm_token[pb] = static_cast<int32_t>(t);
@@ -409,6 +425,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
   uint4* dst = reinterpret_cast<uint4*>(xp);
   const int64_t total = 2 * kRouteTokens * vec_per_row;
   const int64_t stride = static_cast<int64_t>(blockDim.x) * gridDim.y;
+  uint32_t f16_bad = 0;
   for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; i0 < total; i0 += 8 * stride) {
     uint4 v[8];
     int64_t o[8];
@@ -427,9 +444,18 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (o[u] >= 0) dst[o[u]] = F16 ? bf16x8_to_f16x8(v[u]) : v[u];
+    for (int u = 0; u < 8; ++u) {
+      if (o[u] < 0) continue;
+      if (F16) {
+        const uint4 h = bf16x8_to_f16x8(v[u]);
+        f16_bad |= f16x8_nonfinite(h);
+        dst[o[u]] = h;
+      } else {
+        dst[o[u]] = v[u];
+      }
+    }
   }
+  if (F16 && f16_bad) atomicOr(status, kStatusFp16Range);
 }
 
 template <typename TO>
@@ -453,7 +479,8 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 template <typename TO>
 __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ y, int64_t split_stride,
                                                           int32_t splits, const int32_t* __restrict__ slot_pos,
-                                                          int64_t T, int64_t d, TO* __restrict__ out) {
+                                                          int64_t T, int64_t d, TO* __restrict__ out,
+                                                          uint32_t* __restrict__ status) {
   const int64_t q = d / 4;
   const int64_t n = T * q;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -469,6 +496,10 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
         const int64_t c = (i - t * q) * 4;
         const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (kDebugBounds && !(index_ok(p0, 2 * T) && index_ok(p1, 2 * T))) {
+          atomicOr(status, kStatusBounds);
+          continue;
+        }
         for (int s = 0; s < splits; ++s) {
           const float4 uu = *reinterpret_cast<const float4*>(y + s * split_stride + p0 * d + c);
           const float4 vv = *reinterpret_cast<const float4*>(y + s * split_stride + p1 * d + c);
@@ -514,10 +545,15 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(const float* __re
                                                                int32_t splits, const int32_t* __restrict__ slot_pos,
                                                                int64_t d, const TO* __restrict__ residual,
                                                                const float* __restrict__ norm_weight, float eps,
-                                                               TO* __restrict__ out) {
+                                                               TO* __restrict__ out, uint32_t* __restrict__ status) {
   __shared__ float red[8];
   const int64_t t = blockIdx.x;
   const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
+  if (kDebugBounds && !(index_ok(p0, 2 * static_cast<int64_t>(gridDim.x)) &&
+                        index_ok(p1, 2 * static_cast<int64_t>(gridDim.x)))) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusBounds);
+    return;  // uniform over the CTA: one token row per CTA
+  }
   auto row_y = [&](int64_t c) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     for (int s = 0; s < splits; ++s) {
@@ -592,7 +628,7 @@ cudaError_t launch_router(moe_dtype_t dtype, const void* x, const float* w_route
 cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t d, int64_t nblk,
                             const int32_t* idx, const float* gates, const int32_t* hist, int32_t* hist_pre,
                             int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
-                            int32_t* slot_pos, float* gate_perm, void* xp, cudaStream_t s) {
+                            int32_t* slot_pos, float* gate_perm, void* xp, uint32_t* status, cudaStream_t s) {
   // Many router blocks: scan their histograms once (hist_pre holds nblk * E
   // prefixes followed by E totals); few: each dispatch CTA sums them itself.
   const int32_t* pre = nullptr;
@@ -611,40 +647,137 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
   if (dtype == MOE_F32)
     moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(
         static_cast<const float*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
-        slot_pos, gate_perm, static_cast<float*>(xp), pre, tot);
+        slot_pos, gate_perm, static_cast<float*>(xp), pre, tot, status);
   else if (dtype == MOE_BF16_INT8W)
     moe_dispatch_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
-        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot);
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
   else
     moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
-        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot);
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
                            const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
-                           const float* norm_weight, float norm_eps, void* out, cudaStream_t s) {
+                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s) {
   if (residual || norm_weight) {
     if (dtype == MOE_F32)
       moe_combine_norm_kernel<float><<<static_cast<unsigned>(T), 256, 0, s>>>(
           y, split_stride, splits, slot_pos, d, static_cast<const float*>(residual), norm_weight, norm_eps,
-          static_cast<float*>(out));
+          static_cast<float*>(out), status);
     else
       moe_combine_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, 0, s>>>(
           y, split_stride, splits, slot_pos, d, static_cast<const __nv_bfloat16*>(residual), norm_weight,
-          norm_eps, static_cast<__nv_bfloat16*>(out));
+          norm_eps, static_cast<__nv_bfloat16*>(out), status);
     return cudaGetLastError();
   }
   const int64_t n = T * (d / 4);
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(device_sm_count()) * 8);
   if (dtype == MOE_F32)
     moe_combine_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(y, split_stride, splits, slot_pos, T,
-                                                                           d, static_cast<float*>(out));
+                                                                           d, static_cast<float*>(out), status);
   else
     moe_combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        y, split_stride, splits, slot_pos, T, d, static_cast<__nv_bfloat16*>(out));
+        y, split_stride, splits, slot_pos, T, d, static_cast<__nv_bfloat16*>(out), status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Pieces of the expert-parallel form (experts split over GPUs, token rows
+// exchanged between them); see moe_experts_forward and moe_gather_rows.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+// One CTA: counts of the n local experts into the kE slots the GEMM kernels
+// schedule from (slots past n get no rows), their exclusive offsets, and 1.0
+// into `ones` (gates of rows that carry none).
+__global__ void moe_local_schedule_kernel(const int32_t* __restrict__ counts_in, int32_t n,
+                                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                          float* __restrict__ ones, int64_t n_ones) {
+  if (threadIdx.x == 0) {
+    int32_t off = 0;
+    for (int e = 0; e < kE; ++e) {
+      const int32_t c = e < n ? counts_in[e] : 0;
+      counts[e] = c;
+      offsets[e] = off;
+      off += c;
+    }
+    offsets[kE] = off;
+  }
+  if (ones != nullptr)
+    for (int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.x) * blockDim.x; i < n_ones;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      ones[i] = 1.0f;
+}
+
+// y[i] = sum over s of part[s][i], s ascending from 0 (fixed order).
+__global__ void __launch_bounds__(256) moe_sum_splits_kernel(const float* __restrict__ part, int64_t split_stride,
+                                                             int32_t splits, int64_t n4, float* __restrict__ y) {
+  for (int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.x) * blockDim.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+      const float4 v = reinterpret_cast<const float4*>(part + s * split_stride)[i];
+      a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    }
+    reinterpret_cast<float4*>(y)[i] = a;
+  }
+}
+
+// dst row i = src row index[i]; rows of `vecs` vectors of type V (16 or 4 bytes).
+template <typename V>
+__global__ void __launch_bounds__(256) moe_gather_rows_kernel(const V* __restrict__ src, int64_t src_rows,
+                                                              const int32_t* __restrict__ index, int64_t n,
+                                                              int64_t vecs, V* __restrict__ dst,
+                                                              uint32_t* __restrict__ status) {
+  const int64_t total = n * vecs;
+  for (int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.x) * blockDim.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vecs, c = i - r * vecs;
+    const int64_t from = index[r];
+    if (kDebugBounds && !index_ok(from, src_rows)) {
+      atomicOr(status, kStatusBounds);
+      continue;
+    }
+    dst[i] = src[from * vecs + c];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_local_schedule(const int32_t* counts_in, int32_t n, int32_t* counts, int32_t* offsets,
+                                  float* ones, int64_t n_ones, cudaStream_t s) {
+  const int64_t blocks = ones ? std::min<int64_t>(std::max<int64_t>(1, (n_ones + 255) / 256), 1024) : 1;
+  moe_local_schedule_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(counts_in, n, counts, offsets, ones,
+                                                                          n_ones);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sum_splits(const float* part, int64_t split_stride, int32_t splits, int64_t n, float* y,
+                              cudaStream_t s) {
+  const int64_t n4 = n / 4;
+  const int64_t blocks = std::min<int64_t>(std::max<int64_t>(1, (n4 + 255) / 256), device_sm_count() * 8);
+  moe_sum_splits_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(part, split_stride, splits, n4, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* src, int64_t src_rows, const int32_t* index, int64_t n,
+                               int64_t row_bytes, void* dst, uint32_t* status, cudaStream_t s) {
+  // 16-byte vectors when the rows allow them, else 4-byte words.
+  const bool wide = row_bytes % 16 == 0;
+  const int64_t vecs = row_bytes / (wide ? 16 : 4);
+  const int64_t blocks = std::min<int64_t>(std::max<int64_t>(1, (n * vecs + 255) / 256), device_sm_count() * 8);
+  if (wide)
+    moe_gather_rows_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const uint4*>(src), src_rows, index, n, vecs, static_cast<uint4*>(dst), status);
+  else
+    moe_gather_rows_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const uint32_t*>(src), src_rows, index, n, vecs, static_cast<uint32_t*>(dst), status);
   return cudaGetLastError();
 }
 

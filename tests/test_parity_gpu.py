@@ -386,6 +386,42 @@ def test_int8_tall_tiles_both_halves(T, skew):
     full_check(inp, g)
 
 
+def _status_after(inp, x, path=moe.MOE_PATH_AUTO):
+    T, d = x.shape
+    f = inp["w_gate"].shape[2]
+    ws = torch.empty(moe.moe_workspace_size(T, d, f, dtype=moe.MOE_BF16_INT8W, path=path), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.empty_like(x)
+    moe.moe_forward_ex(x, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"], out, ws,
+                       scales=(inp["s_gate"], inp["s_up"], inp["s_down"]), path=path)
+    return moe.moe_device_status(ws)
+
+
+@pytest.mark.parametrize("path", [moe.MOE_PATH_WEIGHT_STREAM, moe.MOE_PATH_TOKEN_TILE_SINGLE])
+def test_int8_fp16_range_is_reported(path):
+    # The int8-weight GEMMs take fp16 operands: a bf16 activation above 65504
+    # in magnitude, or a GeGLU intermediate that large, cannot be represented.
+    # The library flags it (status bit 0x20) instead of returning a silently
+    # wrong output. An ordinary finite input triggers it; nothing faults.
+    inp = small_bf16(300, seed=120, int8=True)
+    assert _status_after(inp, inp["x"], path) == (0, 0)
+    x = inp["x"].clone()
+    x[150, 7] = 1e5                                   # finite in bf16, not in fp16
+    st, code = _status_after(inp, x, path)
+    assert st == moe.N.MOE_ERR_DEVICE_CHECK and code == 0x20
+    # H overflow with in-range activations: unit scales and every code 127 make
+    # x . w_gate about 127 * sqrt(d) * 4, so GELU(gate) * up is far above 65504.
+    big = dict(inp)
+    for w in ("w_gate", "w_up"):
+        big[w] = torch.full_like(inp[w], 127)
+    for s_ in ("s_gate", "s_up"):
+        big[s_] = torch.ones_like(inp[s_])
+    xs = torch.full_like(inp["x"], 4.0)
+    st, code = _status_after(big, xs, path)
+    assert st == moe.N.MOE_ERR_DEVICE_CHECK and code == 0x20
+    assert _status_after(inp, inp["x"], path) == (0, 0)  # the next call starts clean
+
+
 @pytest.mark.parametrize("splits", [2, 3])
 def test_int8_token_tile_split_k(splits):
     inp = small_bf16(600, d=512, f=384, seed=91, int8=True)
