@@ -257,12 +257,26 @@ __device__ __forceinline__ void convert_int8_segment(const uint8_t* w8, uint8_t*
 // per (slot, K split), each produced by a different tile (the two slots are
 // different experts). Every piece is stored in Y[split, permuted row] by the
 // epilogue that produced it, which then counts itself on the arrival counter
-// of (t, column tile) after a fence. The epilogue whose arrival completes the
-// count (it never waits: everything it needs is already in memory) sums the
-// pieces in a fixed order, slot 0 over splits, then slot 1 over splits, then
-// the two, adds the residual row if any, and stores the bf16 output: the result
-// does not depend on which tile finished last, and no output is updated with
-// atomics.
+// of (t, column tile) with a release-acquire atomic add. The epilogue whose
+// arrival completes the count (it never waits: everything it needs is already
+// in memory) sums the pieces in a fixed order, slot 0 over splits, then slot 1
+// over splits, then the two, adds the residual row if any, and stores the bf16
+// output: the result does not depend on which tile finished last, and no
+// output is updated with atomics. The pieces are dead once summed, so their L2
+// lines are dropped without being written back to DRAM.
+
+// Counter add with release (this thread's piece is visible device-wide before
+// the count) and acquire (the pieces counted before are visible after it).
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Invalidate one 128-byte L2 line without writing it back (its data is dead).
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 
 // Fixed-order sum of the 2 * splits pieces of token `tok`, columns n0 + 8 * lane
 // .. + 7, read from L2 (other SMs wrote them), stored as bf16.
@@ -302,6 +316,15 @@ __device__ __forceinline__ void combine_columns(const Params& p, int tok, int n0
   }
   *reinterpret_cast<uint4*>(p.combine_out + at) =
       make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+  // Every lane has its values (they were summed above); then one lane per
+  // 128-byte line drops the line: four lanes read 32 bytes each of it.
+  __syncwarp();
+  if ((lane & 3) == 0) {
+    for (int s = 0; s < p.splits; ++s) {
+      discard_l2_line(y + s * p.split_stride + p0 * p.N + c);
+      discard_l2_line(y + s * p.split_stride + p1 * p.N + c);
+    }
+  }
 }
 
 // Called by a whole epilogue warp after each lane stored its row's piece of
@@ -320,13 +343,15 @@ __device__ __forceinline__ void combine_arrive(const Params& p, const Tile& t, i
     }
   }
   if (valid) {
-    __threadfence();  // this lane's piece is visible device-wide before it is counted
-    const int old = atomicAdd(&p.combine_count[static_cast<int64_t>(tok) * (p.N / 256) + t.n0 / 256], 1);
+    const int old =
+        atomic_add_acq_rel_gpu(&p.combine_count[static_cast<int64_t>(tok) * (p.N / 256) + t.n0 / 256], 1);
     last = old == 2 * p.splits - 1;
   }
   unsigned m = __ballot_sync(0xffffffffu, last);
   if (m == 0) return;
-  __threadfence();  // the counted pieces of other SMs are read after the count
+  // Warp barrier: what the acquiring lanes observed is visible to every lane
+  // that reads the pieces below.
+  __syncwarp();
   const int lane = threadIdx.x % 32;
   while (m) {
     const int src = __ffs(m) - 1;

@@ -57,12 +57,18 @@ constexpr int XBOX_ROWS_WS = 32;        // WEIGHT_STREAM activation box height
 // columns 0-255, rows 128-255 into 256-511), so the conversion and the converted
 // tile's shared-memory traffic per FLOP halve. The two halves of TMEM then hold
 // one tile, and the epilogue no longer overlaps the next tile's main loop.
-template <bool W8, bool TALL = false>
+// SHORT (weight-stream tiles of at most 64 tokens, for small batches): the
+// activation box of a slot shrinks to 8 KB, so the ring holds more weight
+// stages in flight (int8: 6 slots = 96 KB of int8 weights instead of 4 = 64 KB;
+// bf16: 5 slots = 160 KB instead of 128 KB). A weight-stream kernel streams
+// every weight byte once with little reuse, so the bytes in flight per SM set
+// its bandwidth.
+template <bool W8, bool TALL = false, bool SHORT = false>
 struct Cfg {
-  static constexpr int XS_BYTES = (TALL ? 2 : 1) * X_BYTES;
-  static constexpr int STAGES = TALL ? 3 : 4;
+  static constexpr int XS_BYTES = SHORT ? 64 * 128 : (TALL ? 2 : 1) * X_BYTES;
+  static constexpr int STAGES = SHORT ? (W8 ? 6 : 5) : (TALL ? 3 : 4);
   static constexpr int SLOT_BYTES = XS_BYTES + (W8 ? W8_BYTES : W_BYTES);
-  static constexpr int CSTAGES = W8 ? (TALL ? 2 : 3) : 0;
+  static constexpr int CSTAGES = W8 ? ((TALL || SHORT) ? 2 : 3) : 0;
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
@@ -71,21 +77,25 @@ struct Cfg {
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
 constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ring
-static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages,
+static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages &&
+                  Cfg<true, false, true>::CSTAGES <= kMaxCStages,
               "converted-W ring deeper than its barrier slots");
-static_assert((2 * Cfg<true>::STAGES + 2 * kMaxCStages + 4) * 8 + 16 + sizeof(SharedSched) <= Cfg<true>::BAR_BYTES,
+static_assert((2 * Cfg<true, false, true>::STAGES + 2 * kMaxCStages + 4) * 8 + 16 + sizeof(SharedSched) <=
+                  Cfg<true>::BAR_BYTES,
               "barrier area too small");
-static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cfg<false>::SMEM <= 232448,
+static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cfg<false>::SMEM <= 232448 &&
+                  Cfg<true, false, true>::SMEM <= 232448 && Cfg<false, false, true>::SMEM <= 232448,
               "shared memory above the per-block limit");
 
-template <int KIND, bool WS, bool W8>
+template <int KIND, bool WS, bool W8, bool SHORT = false>
 __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     moe_expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                            const __grid_constant__ CUtensorMap tm_w1, const Params p) {
+  static_assert(!SHORT || WS, "short tiles are a weight-stream form");
   constexpr bool TALL = W8 && !WS;
-  constexpr int TROWS = TALL ? 2 * BM : BM;  // token rows per tile
+  constexpr int TROWS = TALL ? 2 * BM : (SHORT ? BM / 2 : BM);  // token rows per tile
   constexpr int NACC = TALL ? 1 : 2;         // accumulator buffers in flight
-  using C = Cfg<W8, TALL>;
+  using C = Cfg<W8, TALL, SHORT>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-B swizzle atoms.
@@ -260,7 +270,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           }
           tc_fence_after();
           const uint32_t xs = smem_u32(smem + stage * C::SLOT_BYTES);
-          const uint32_t ws = W8 ? smem_u32(conv_area + cstage * W_BYTES) : xs + X_BYTES;
+          const uint32_t ws = W8 ? smem_u32(conv_area + cstage * W_BYTES) : xs + C::XS_BYTES;
           const bool second_half = TALL && t.rows > BM;  // rows 128..255 of a tall tile
 #pragma unroll
           for (int k16 = 0; k16 < BK / 16; ++k16) {
@@ -433,11 +443,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   }
 }
 
-template <int KIND, bool WS, bool W8>
+template <int KIND, bool WS, bool W8, bool SHORT = false>
 cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   constexpr bool TALL = W8 && !WS;
-  using C = Cfg<W8, TALL>;
-  auto kern = moe_expert_gemm_kernel<KIND, WS, W8>;
+  using C = Cfg<W8, TALL, SHORT>;
+  auto kern = moe_expert_gemm_kernel<KIND, WS, W8, SHORT>;
   const cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
 
@@ -494,7 +504,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.residual = fuse ? static_cast<const __nv_bfloat16*>(a.residual) : nullptr;
 
   // Upper bound of the tile count (the exact count is only known on device).
-  const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : BM) + kE;
+  const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : (SHORT ? BM / 2 : BM)) + kE;
   const int64_t tiles_max = mtiles_max * (a.N / p.ntile) * p.splits;
   const int grid = static_cast<int>(std::min<int64_t>(tiles_max, device_sm_count()));
   kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_x, tm_w0, tm_w1, p);
@@ -504,12 +514,18 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
 }  // namespace tc
 
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s) {
+  if (a.weight_stream && a.short_tiles)
+    return a.int8_weights ? tc::launch_one<tc::GATEUP, true, true, true>(a, s)
+                          : tc::launch_one<tc::GATEUP, true, false, true>(a, s);
   if (a.weight_stream)
     return a.int8_weights ? tc::launch_one<tc::GATEUP, true, true>(a, s) : tc::launch_one<tc::GATEUP, true, false>(a, s);
   return a.int8_weights ? tc::launch_one<tc::GATEUP, false, true>(a, s) : tc::launch_one<tc::GATEUP, false, false>(a, s);
 }
 
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s) {
+  if (a.weight_stream && a.short_tiles)
+    return a.int8_weights ? tc::launch_one<tc::DOWN, true, true, true>(a, s)
+                          : tc::launch_one<tc::DOWN, true, false, true>(a, s);
   if (a.weight_stream)
     return a.int8_weights ? tc::launch_one<tc::DOWN, true, true>(a, s) : tc::launch_one<tc::DOWN, true, false>(a, s);
   return a.int8_weights ? tc::launch_one<tc::DOWN, false, true>(a, s) : tc::launch_one<tc::DOWN, false, false>(a, s);

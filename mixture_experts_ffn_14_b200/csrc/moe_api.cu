@@ -371,6 +371,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.act = o->activation;
     g.int8_weights = w8;
     g.weight_stream = L.weight_stream;
+    // Small batches (<= 32 token slots per expert on average): weight-stream
+    // tiles of at most 64 tokens, which leave room for more weight stages in flight.
+    g.short_tiles = L.weight_stream && T <= 128;
     g.status = status;
     g.tile_counter = tile_counters;
     // Token tiles: with MOE_PATH_AUTO both forms are launched and the kernels
@@ -772,6 +775,7 @@ moe_status_t moe_experts_forward(const moe_expert_rows_t* a, const moe_options_t
   g.act = o->activation;
   g.int8_weights = w8;
   g.weight_stream = L.weight_stream;
+  g.short_tiles = L.weight_stream && R <= 32 * static_cast<int64_t>(a->n_experts);
   g.status = status;
   g.n_experts = a->n_experts;
   // One token-tile form per call here (the single-CTA one unless the pair form

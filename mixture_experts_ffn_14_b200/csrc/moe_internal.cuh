@@ -119,6 +119,7 @@ struct TcGemmArgs {
   int32_t* tile_counter;    // pair form: zeroed int that hands out tiles in order, or nullptr (static order)
   uint32_t* status;
   int32_t n_experts;        // experts in the weight arrays (0 = kE); experts past it have no rows
+  bool short_tiles;         // weight-stream: tiles of at most 64 tokens, deeper weight ring
   // DOWN token tiles: the combine in the epilogue (out[t] = sum of the two
   // gate-scaled rows of token t, in fixed order). combine_count == nullptr:
   // the epilogue only writes Y and a separate combine kernel runs.

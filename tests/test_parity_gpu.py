@@ -373,6 +373,19 @@ def test_int8_tile_boundaries(T):
         full_check(inp, gpu)
 
 
+@pytest.mark.parametrize("int8", [False, True])
+@pytest.mark.parametrize("T", [64, 65, 100, 128])
+def test_weight_stream_short_tiles_split_an_expert(T, int8):
+    # Batches of at most 128 tokens take weight-stream tiles of at most 64
+    # tokens; with every token on experts 0 and 1 those experts need one or two
+    # tiles each (64 = one full tile, 65 = a full one and a single-token one).
+    inp = small_bf16(T, seed=130 + T, int8=int8)
+    inp["router_bias"] = torch.tensor([40.0, 30.0, 0, 0, 0, 0, 0, 0], device=DEV)
+    gpu = run_gpu(inp)
+    assert list(gpu["counts"][:2]) == [T, T]
+    full_check(inp, gpu)
+
+
 @pytest.mark.parametrize("T,skew", [(516, False), (1028, False), (700, True)])
 def test_int8_tall_tiles_both_halves(T, skew):
     # int8 token tiles hold 256 rows as two MMAs on one converted weight tile;
