@@ -375,6 +375,21 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
     uint32_t f16_bad = 0;  // int8 weights: an H value beyond the fp16 range
 #pragma unroll 1
     for (int c = 0; c < 128; c += 32) {
+      // int8 weights: the chunk's 32 gate and 32 up channel scales as eight
+      // 16-byte loads (the same addresses in every lane), issued before the
+      // TMEM load so that their latency overlaps it.
+      uint32_t sg[16], su[16];
+      if (W8) {
+        const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c;
+        const uint4* a = reinterpret_cast<const uint4*>(p.s0 + sc);
+        const uint4* b = reinterpret_cast<const uint4*>(p.s1 + sc);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = __ldg(a + v), y = __ldg(b + v);
+          sg[4 * v] = x.x; sg[4 * v + 1] = x.y; sg[4 * v + 2] = x.z; sg[4 * v + 3] = x.w;
+          su[4 * v] = y.x; su[4 * v + 1] = y.y; su[4 * v + 2] = y.z; su[4 * v + 3] = y.w;
+        }
+      }
       uint32_t g[32], u[32];
       tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
       uint32_t packed[16];
@@ -382,12 +397,11 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
       for (int j = 0; j < 32; j += 2) {
         float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
         float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
-        if (W8) {
-          const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c + j;
-          g0 *= __bfloat162float(p.s0[sc]);
-          g1 *= __bfloat162float(p.s0[sc + 1]);
-          u0 *= __bfloat162float(p.s1[sc]);
-          u1 *= __bfloat162float(p.s1[sc + 1]);
+        if (W8) {  // bf16 pair (lo = column j, hi = j + 1) -> fp32 by a shift
+          g0 *= __uint_as_float(sg[j / 2] << 16);
+          g1 *= __uint_as_float(sg[j / 2] & 0xFFFF0000u);
+          u0 *= __uint_as_float(su[j / 2] << 16);
+          u1 *= __uint_as_float(su[j / 2] & 0xFFFF0000u);
         }
         // int8 weights run the MMAs on fp16 operands, so H is stored as fp16 there.
         const float h0 = act_f32(g0, p.act) * u0, h1 = act_f32(g1, p.act) * u1;
@@ -407,6 +421,15 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
     const float gate = valid ? p.gate_perm[row] : 0.0f;
 #pragma unroll 1
     for (int c = 0; c < 256; c += 32) {
+      uint32_t sd[16];  // int8 weights: the chunk's 32 channel scales (four 16-byte loads)
+      if (W8) {
+        const uint4* a = reinterpret_cast<const uint4*>(p.s0 + static_cast<int64_t>(t.e) * p.N + t.n0 + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 x = __ldg(a + q);
+          sd[4 * q] = x.x; sd[4 * q + 1] = x.y; sd[4 * q + 2] = x.z; sd[4 * q + 3] = x.w;
+        }
+      }
       uint32_t v[32];
       tmem_ld32(tbase + c, v);
       if (valid) {
@@ -414,7 +437,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float a = __uint_as_float(v[j]);
-          if (W8) a *= __bfloat162float(p.s0[static_cast<int64_t>(t.e) * p.N + t.n0 + c + j]);
+          if (W8) a *= __uint_as_float((j & 1) ? (sd[j / 2] & 0xFFFF0000u) : (sd[j / 2] << 16));
           o[j] = a * gate;
         }
         float4* dst = reinterpret_cast<float4*>(yout + row * p.N + t.n0 + c);

@@ -77,11 +77,21 @@ struct Cfg {
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
 constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ring
+// Token tiles hand out their tiles in order from a global counter (zeroed by
+// the caller) when one is given: the producer takes the next tile id when it
+// starts a tile and passes it through a queue of kTileQS slots to the other
+// roles (MMA thread, epilogue warps, converter warps), which read the tiles
+// in the same order. A CTA that finishes early takes more tiles instead of
+// idling (the tiles of one call differ in cost: short last row tiles, tall
+// int8 tiles with one or two MMAs per step), and consecutive tile ids (the row
+// tiles that share one weight tile) go to CTAs that became free together, so
+// they read that weight tile from L2 close in time.
+constexpr int kTileQS = 4;
 static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages &&
                   Cfg<true, false, true>::CSTAGES <= kMaxCStages,
               "converted-W ring deeper than its barrier slots");
-static_assert((2 * Cfg<true, false, true>::STAGES + 2 * kMaxCStages + 4) * 8 + 16 + sizeof(SharedSched) <=
-                  Cfg<true>::BAR_BYTES,
+static_assert((2 * Cfg<true, false, true>::STAGES + 2 * kMaxCStages + 4 + 2 * kTileQS) * 8 + 16 +
+                      sizeof(SharedSched) + 4 * kTileQS <= Cfg<true>::BAR_BYTES,
               "barrier area too small");
 static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cfg<false>::SMEM <= 232448 &&
                   Cfg<true, false, true>::SMEM <= 232448 && Cfg<false, false, true>::SMEM <= 232448,
@@ -108,9 +118,12 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   uint64_t* cempty_bar = cfull_bar + kMaxCStages;               // converted W slot free again
   uint64_t* tfull_bar = cempty_bar + kMaxCStages;
   uint64_t* tempty_bar = tfull_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  uint64_t* qfull_bar = tempty_bar + 2;        // tile-id queue slot written
+  uint64_t* qempty_bar = qfull_bar + kTileQS;  // tile-id queue slot read by every consumer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty_bar + kTileQS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   SharedSched* sched = reinterpret_cast<SharedSched*>(tmem_slot + 4);
+  volatile int* tile_q = reinterpret_cast<volatile int*>(sched + 1);
 
   if (skip_launch(p)) return;  // the other token-tile form takes this call
 
@@ -131,8 +144,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 128);
     }
+    for (int i = 0; i < kTileQS; ++i) {
+      mbar_init(&qfull_bar[i], 1);
+      mbar_init(&qempty_bar[i], 1 + 4 + (W8 ? C::CONVERT_WARPS : 0));  // MMA, epilogue warps, converter warps
+    }
     *abort_flag = 0;
-    build_sched(*sched, p, TROWS);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -144,10 +160,48 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  // Weight-stream launches follow the previous kernel with programmatic
+  // serialisation: the set-up above overlaps its last CTAs, the counts and
+  // rows it produced are read only past this wait.
+  pdl_wait();
+  if (threadIdx.x == 0) build_sched(*sched, p, TROWS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
+
+  // ---- tile order (see kTileQS). Queue operations return the tile id, -1
+  // when no tile is left, -2 when a wait timed out.
+  const bool dyn = !WS && p.tile_counter != nullptr;
+  const int ntiles = sched->pre[kE];
+  auto q_fill = [&](int i) -> int {  // producer, lane 0
+    const int slot = i % kTileQS;
+    const uint32_t ph = (i / kTileQS) & 1;
+    if (!mbar_wait(&qempty_bar[slot], ph ^ 1, kWaitLimitNs) || *abort_flag) return -2;
+    const int t = atomicAdd(p.tile_counter, 1);
+    const int tile = t < ntiles ? t : -1;
+    tile_q[slot] = tile;
+    mbar_arrive(&qfull_bar[slot]);
+    return tile;
+  };
+  auto q_take = [&](int i) -> int {  // the MMA thread
+    const int slot = i % kTileQS;
+    const uint32_t ph = (i / kTileQS) & 1;
+    if (!mbar_wait(&qfull_bar[slot], ph, kWaitLimitNs) || *abort_flag) return -2;
+    const int tile = tile_q[slot];
+    mbar_arrive(&qempty_bar[slot]);
+    return tile;
+  };
+  auto q_take_warp = [&](int i) -> int {  // a whole epilogue or converter warp, one arrive
+    const int slot = i % kTileQS;
+    const uint32_t ph = (i / kTileQS) & 1;
+    if (!warp_wait(&qfull_bar[slot], ph, abort_flag)) return -2;
+    const int tile = tile_q[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qempty_bar[slot]);
+    return tile;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -168,7 +222,20 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
+      for (int i = 0;; ++i) {
+        int tile = blockIdx.x + i * gridDim.x;
+        if (dyn) {
+          if (!G || lane == 0) tile = q_fill(i);
+          if (G) tile = __shfl_sync(0xffffffffu, tile, 0);
+          if (tile == -2) {
+            if (!G || lane == 0) {
+              atomicOr(p.status, kStatusProducerTimeout);
+              *abort_flag = 1;
+            }
+            return;
+          }
+        }
+        if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
         int32_t rtok[4] = {0, 0, 0, 0};
         if (G) gather_rows(p, t, t.row0 + 4 * lane, rtok);
         const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
@@ -246,7 +313,14 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       Tile t;
-      for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
+      for (int i = 0;; ++i) {
+        const int tile = dyn ? q_take(i) : static_cast<int>(blockIdx.x + i * gridDim.x);
+        if (tile == -2) {
+          atomicOr(p.status, kStatusMmaTimeout);
+          *abort_flag = 1;
+          goto mma_done;
+        }
+        if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, kWaitLimitNs) || *abort_flag) {
           atomicOr(p.status, kStatusMmaTimeout);
           *abort_flag = 1;
@@ -319,7 +393,14 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
+    for (int i = 0;; ++i) {
+      const int tile = dyn ? q_take_warp(i) : static_cast<int>(blockIdx.x + i * gridDim.x);
+      if (tile == -2) {
+        atomicOr(p.status, kStatusEpilogueTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
       if (!warp_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         atomicOr(p.status, kStatusEpilogueTimeout);
         *abort_flag = 1;
@@ -402,7 +483,14 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     int cstage = 0;
     uint32_t cphase = 0;
     Tile t;
-    for (int tile = blockIdx.x; decode_tile(*sched, p, tile, TROWS, t); tile += gridDim.x) {
+    for (int i = 0;; ++i) {
+      const int tile = dyn ? q_take_warp(i) : static_cast<int>(blockIdx.x + i * gridDim.x);
+      if (tile == -2) {
+        atomicOr(p.status, kStatusConvertTimeout);
+        *abort_flag = 1;
+        goto convert_done;
+      }
+      if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
       for (int kb = 0; kb < p.kb_per_split; ++kb) {
         if (!warp_wait(&full_bar[stage], phase, abort_flag) || !warp_wait(&cempty_bar[cstage], cphase ^ 1, abort_flag)) {
           atomicOr(p.status, kStatusConvertTimeout);
@@ -481,7 +569,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.offsets = a.offsets;
   p.gate_perm = a.gate_perm;
   p.row_token = (!WS && KIND == GATEUP) ? a.row_token : nullptr;
-  p.tile_counter = nullptr;  // static tile order
+  p.tile_counter = WS ? nullptr : a.tile_counter_single;  // token tiles: dynamic order when given
   p.s0 = a.s0;
   p.s1 = a.s1;
   p.out = a.out;
@@ -507,6 +595,8 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : (SHORT ? BM / 2 : BM)) + kE;
   const int64_t tiles_max = mtiles_max * (a.N / p.ntile) * p.splits;
   const int grid = static_cast<int>(std::min<int64_t>(tiles_max, device_sm_count()));
+  if (WS)  // decode-sized batches: behind the dispatch / gate-up kernel (see pdl_wait)
+    return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, stream, tm_x, tm_w0, tm_w1, p);
   kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_x, tm_w0, tm_w1, p);
   return cudaGetLastError();
 }

@@ -297,8 +297,9 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
-  // Tile counters of the two CTA-pair GEMM launches, in the status slot (zeroed
-  // with it below).
+  // Tile counters of the token-tile GEMM launches (pair gate/up, pair down,
+  // single-CTA gate/up, single-CTA down), in the status slot (zeroed with it
+  // below).
   int32_t* tile_counters = reinterpret_cast<int32_t*>(ws + L.status + 16);
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
   float* gates = reinterpret_cast<float*>(ws + L.gates);
@@ -376,6 +377,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.short_tiles = L.weight_stream && T <= 128;
     g.status = status;
     g.tile_counter = tile_counters;
+    g.tile_counter_single = tile_counters + 2;
     // Token tiles: with MOE_PATH_AUTO both forms are launched and the kernels
     // pick one of them on the device from the expert counts (the other returns
     // at once); TOKEN_TILE / TOKEN_TILE_SINGLE force one form.
@@ -411,6 +413,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g2.N = static_cast<int32_t>(d);
     g2.splits = L.splits;
     g2.tile_counter = tile_counters + 1;
+    g2.tile_counter_single = tile_counters + 3;
     if (fused_combine) {
       g2.perm_token = perm_token;
       g2.slot_pos = slot_pos;
@@ -819,7 +822,7 @@ moe_status_t moe_combine(const float* y, const int32_t* slot_pos, int64_t T, int
   uint32_t* status = static_cast<uint32_t*>(workspace);
   if (cudaMemsetAsync(status, 0, kAlign, s) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_combine(dtype, y, 2 * T * d, 1, slot_pos, T, d, residual, post_norm_weight, norm_eps, out, status,
-                        s) == cudaSuccess
+                        s, /*pdl=*/false) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
