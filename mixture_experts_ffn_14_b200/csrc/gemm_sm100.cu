@@ -160,15 +160,10 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // Weight-stream launches follow the previous kernel with programmatic
-  // serialisation: the set-up above overlaps its last CTAs, the counts and
-  // rows it produced are read only past this wait.
-  pdl_wait();
   if (threadIdx.x == 0) build_sched(*sched, p, TROWS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_launch_dependents();
   const uint32_t tmem_base = *tmem_slot;
 
   // ---- tile order (see kTileQS). Queue operations return the tile id, -1
@@ -595,8 +590,6 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   const int64_t mtiles_max = a.rows / (TALL ? 2 * BM : (SHORT ? BM / 2 : BM)) + kE;
   const int64_t tiles_max = mtiles_max * (a.N / p.ntile) * p.splits;
   const int grid = static_cast<int>(std::min<int64_t>(tiles_max, device_sm_count()));
-  if (WS)  // decode-sized batches: behind the dispatch / gate-up kernel (see pdl_wait)
-    return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, stream, tm_x, tm_w0, tm_w1, p);
   kern<<<grid, C::THREADS, C::SMEM, stream>>>(tm_x, tm_w0, tm_w1, p);
   return cudaGetLastError();
 }

@@ -822,7 +822,7 @@ moe_status_t moe_combine(const float* y, const int32_t* slot_pos, int64_t T, int
   uint32_t* status = static_cast<uint32_t*>(workspace);
   if (cudaMemsetAsync(status, 0, kAlign, s) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_combine(dtype, y, 2 * T * d, 1, slot_pos, T, d, residual, post_norm_weight, norm_eps, out, status,
-                        s, /*pdl=*/false) == cudaSuccess
+                        s) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

@@ -8,49 +8,11 @@
 
 #include <cstddef>
 #include <cstdint>
-#include <utility>
 
 #include "../../include/moe.h"
 #include "bounds.cuh"
 
 namespace moe {
-
-// ---- programmatic dependent launch ----------------------------------------
-// Kernels after the first of a call are launched so that they may start while
-// the previous kernel finishes (its CTAs retire): they set up (barriers, tensor
-// memory) and then wait at pdl_wait() until the previous grid has completed
-// and its writes are visible, before reading anything it produced. Every
-// kernel calls pdl_launch_dependents() once it is past that wait, which lets
-// the next kernel's CTAs be scheduled as SMs free up. Without such a launch
-// both are no-ops.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
-
-// Host: launch `kern` on `s`, with the programmatic-serialisation attribute
-// when `pdl`.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                             Args&&... args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
-// Host: launch `kern` on `s` with the programmatic-serialisation attribute.
-// With pdl == false it is an ordinary launch.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       Args&&... args) {
-  return launch_maybe_pdl(true, kern, grid, block, smem, s, std::forward<Args>(args)...);
-}
 
 constexpr int kE = 8;              // experts (this version)
 constexpr int kK = 2;              // experts per token
@@ -122,12 +84,9 @@ cudaError_t launch_sum_splits(const float* part, int64_t split_stride, int32_t s
 cudaError_t launch_gather_rows(const void* src, int64_t src_rows, const int32_t* index, int64_t n,
                                int64_t row_bytes, void* dst, uint32_t* status, cudaStream_t s);
 
-// pdl: launched with programmatic serialisation behind the previous kernel
-// (false when the previous stream operation is not a kernel).
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
                            const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
-                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s,
-                           bool pdl = true);
+                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s);
 
 // fp32 (SIMT) grouped expert GEMMs.
 cudaError_t launch_f32_gateup(const float* xp, const float* wg, const float* wu, const int32_t* counts,

@@ -323,8 +323,6 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
   __shared__ int pos_sm[kRouteTokens][2];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t blk = blockIdx.x;
-  pdl_wait();  // the router's outputs (or the scan's)
-  pdl_launch_dependents();
 
   // This block's slots start, per expert, after those of all earlier blocks:
   // read from the scan (many blocks) or summed here (few blocks, no extra launch).
@@ -486,8 +484,6 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
   const int64_t q = d / 4;
   const int64_t n = T * q;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  pdl_wait();  // the down projection's rows
-  pdl_launch_dependents();
   // Four outputs per thread per pass, their loads issued before any store.
   for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n; i0 += 4 * stride) {
     float4 r[4];
@@ -552,8 +548,6 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(const float* __re
                                                                TO* __restrict__ out, uint32_t* __restrict__ status) {
   __shared__ float red[8];
   const int64_t t = blockIdx.x;
-  pdl_wait();  // the down projection's rows
-  pdl_launch_dependents();
   const int64_t p0 = slot_pos[2 * t], p1 = slot_pos[2 * t + 1];
   if (kDebugBounds && !(index_ok(p0, 2 * static_cast<int64_t>(gridDim.x)) &&
                         index_ok(p1, 2 * static_cast<int64_t>(gridDim.x)))) {
@@ -650,44 +644,44 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
   const int64_t g =
       xp ? std::min<int64_t>(16, std::max<int64_t>(1, (2 * device_sm_count() + nblk - 1) / nblk)) : 1;
   const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(g), 1);
-  // Launched behind the router (or the scan) with programmatic serialisation:
-  // its CTAs start as the router's retire and wait for its outputs.
   if (dtype == MOE_F32)
-    return launch_pdl(moe_dispatch_kernel<float>, grid, dim3(256), 0, s, static_cast<const float*>(x), T, d, nblk,
-                      idx, gates, hist, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm,
-                      static_cast<float*>(xp), pre, tot, status);
-  if (dtype == MOE_BF16_INT8W)
-    return launch_pdl(moe_dispatch_kernel<__nv_bfloat16, true>, grid, dim3(256), 0, s,
-                      static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets,
-                      perm_token, perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
-  return launch_pdl(moe_dispatch_kernel<__nv_bfloat16, false>, grid, dim3(256), 0, s,
-                    static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
-                    perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
+    moe_dispatch_kernel<float><<<grid, 256, 0, s>>>(
+        static_cast<const float*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token, perm_slot,
+        slot_pos, gate_perm, static_cast<float*>(xp), pre, tot, status);
+  else if (dtype == MOE_BF16_INT8W)
+    moe_dispatch_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
+  else
+    moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
+        perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
                            const int32_t* slot_pos, int64_t T, int64_t d, const void* residual,
-                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s,
-                           bool pdl) {
-  // Launched behind the down projection with programmatic serialisation.
+                           const float* norm_weight, float norm_eps, void* out, uint32_t* status, cudaStream_t s) {
   if (residual || norm_weight) {
-    const dim3 grid(static_cast<unsigned>(T));
     if (dtype == MOE_F32)
-      return launch_maybe_pdl(pdl, moe_combine_norm_kernel<float>, grid, dim3(256), 0, s, y, split_stride, splits, slot_pos, d,
-                        static_cast<const float*>(residual), norm_weight, norm_eps, static_cast<float*>(out),
-                        status);
-    return launch_maybe_pdl(pdl, moe_combine_norm_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, y, split_stride, splits,
-                      slot_pos, d, static_cast<const __nv_bfloat16*>(residual), norm_weight, norm_eps,
-                      static_cast<__nv_bfloat16*>(out), status);
+      moe_combine_norm_kernel<float><<<static_cast<unsigned>(T), 256, 0, s>>>(
+          y, split_stride, splits, slot_pos, d, static_cast<const float*>(residual), norm_weight, norm_eps,
+          static_cast<float*>(out), status);
+    else
+      moe_combine_norm_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, 0, s>>>(
+          y, split_stride, splits, slot_pos, d, static_cast<const __nv_bfloat16*>(residual), norm_weight,
+          norm_eps, static_cast<__nv_bfloat16*>(out), status);
+    return cudaGetLastError();
   }
   const int64_t n = T * (d / 4);
-  const dim3 grid(static_cast<unsigned>(
-      std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(device_sm_count()) * 8)));
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(device_sm_count()) * 8);
   if (dtype == MOE_F32)
-    return launch_maybe_pdl(pdl, moe_combine_kernel<float>, grid, dim3(256), 0, s, y, split_stride, splits, slot_pos, T, d,
-                      static_cast<float*>(out), status);
-  return launch_maybe_pdl(pdl, moe_combine_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, y, split_stride, splits, slot_pos, T,
-                    d, static_cast<__nv_bfloat16*>(out), status);
+    moe_combine_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(y, split_stride, splits, slot_pos, T,
+                                                                           d, static_cast<float*>(out), status);
+  else
+    moe_combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        y, split_stride, splits, slot_pos, T, d, static_cast<__nv_bfloat16*>(out), status);
+  return cudaGetLastError();
 }
 
 }  // namespace moe
