@@ -24,6 +24,10 @@ constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swiz
 constexpr int X_BYTES = BM * BK * 2;    // 16 KB
 constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16, 128-B swizzle
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
+// The producers prefetch the weight boxes of the K block this many stages
+// ahead of the one they load into L2, so that the weight stream's DRAM latency
+// is covered by L2 rather than by the shared-memory ring alone.
+constexpr int kL2PrefetchStages = 8;
 
 enum { GATEUP = 0, DOWN = 1 };
 

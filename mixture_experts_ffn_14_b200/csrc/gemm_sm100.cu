@@ -260,6 +260,22 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
               tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
               if (TALL) tma_load_2d(xs + X_BYTES, &tm_x, &full_bar[stage], k0, t.row0 + BM);
             }
+            // L2 prefetch of the weight boxes kL2PrefetchStages K blocks ahead
+            // (at a tile's first block: of all blocks up to there).
+            for (int ka = kb == 0 ? 1 : kL2PrefetchStages; ka <= kL2PrefetchStages; ++ka) {
+              if (kb + ka >= p.kb_per_split) break;
+              const int kp = k0 + ka * BK;
+              if (W8) {
+                tma_prefetch_l2_3d(&tm_w0, t.n0, kp, t.e);
+                if (KIND == GATEUP) tma_prefetch_l2_3d(&tm_w1, t.n0, kp, t.e);
+                else tma_prefetch_l2_3d(&tm_w0, t.n0 + 128, kp, t.e);
+              } else {
+                for (int j = 0; j < 4; ++j) {
+                  const CUtensorMap* m = (KIND == GATEUP && j >= 2) ? &tm_w1 : &tm_w0;
+                  tma_prefetch_l2_3d(m, t.n0 + 64 * (KIND == GATEUP ? (j & 1) : j), kp, t.e);
+                }
+              }
+            }
             if (W8) {
               if (KIND == GATEUP) {
                 load_w(w8, &tm_w0, &full_bar[stage], t.n0, k0, t.e);
