@@ -342,16 +342,14 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 
 
 def launches_per_step(wl, path):
-    """Kernels of ours per step: router, dispatch, two GEMMs, and a combine
-    kernel on the weight-stream path (token tiles combine in the down
-    projection's epilogue); with the automatic token-tile choice on bf16
-    weights each GEMM launches both forms (the one not chosen returns at once);
-    above 1024 router blocks (T > 32768) a histogram scan runs before the
-    dispatch."""
-    ws = path == "weight_stream" or (path == "auto" and wl.T <= 256)
+    """Kernels of ours per step: router, dispatch and two GEMMs (the down
+    projection's epilogue sums each token's rows, so no combine kernel runs);
+    with the automatic token-tile choice on bf16 weights each GEMM launches both
+    forms (the one not chosen returns at once); above 1024 router blocks
+    (T > 32768) a histogram scan runs before the dispatch."""
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
-    return 4 + (1 if ws else 0) + (2 if both else 0) + (1 if scan else 0)
+    return 4 + (2 if both else 0) + (1 if scan else 0)
 
 
 # ---------------------------------------------------------------- main --
@@ -468,11 +466,11 @@ def main():
         "expert_slots": expert_counts,
         "path": a.path,
         "row_gather": bool(a.row_gather),
-        "combine": "combine kernel" if a.separate_combine else "in the down projection's epilogue (token tiles)",
+        "combine": "combine kernel" if a.separate_combine else "in the down projection's epilogue",
         "hbm_gbs_weights": round(world * K * wbytes / (t_max / 1e3) / 1e9, 1),
         "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": roofline,
-        "gpu_launches": (launches_per_step(wl, a.path) + (1 if a.separate_combine and wl.T > 256 else 0)) * K,
+        "gpu_launches": (launches_per_step(wl, a.path) + (1 if a.separate_combine else 0)) * K,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                    "power_w_max": clocks.get("power_w_max"), "power_w_median": clocks.get("power_w_median"),
                    "samples": clocks.get("samples"), "source": clocks.get("source")},

@@ -156,9 +156,10 @@ typedef struct {
                                   on B200, where four-row gathers cannot feed the MMA).
                                   The weight-stream form always reads the copy;
                                   MOE_BF16_INT8W returns MOE_ERR_UNSUPPORTED with 1.      */
-  int32_t separate_combine;    /* 0: token tiles sum each token's two expert rows in the
-                                  down projection's epilogue (default); 1: a separate
-                                  combine kernel does it (same result bit for bit)       */
+  int32_t separate_combine;    /* 0: the down projection's epilogue sums each token's two
+                                  expert rows (default; bf16 and int8 weights without the
+                                  post-norm); 1: a separate combine kernel does it (same
+                                  result bit for bit)                                     */
 } moe_options_t;
 
 /* Optional outputs for inspection; each is a device pointer or NULL.

@@ -135,7 +135,7 @@ def moe_forward_ex(x, w_router, w_gate, w_up, w_down, out, workspace, scales=Non
     ``row_gather``: token tiles gather their gate/up rows from x with TMA row
     gathers instead of reading the dispatch stage's permuted copy.
     ``separate_combine``: sum each token's two expert rows in a combine kernel
-    instead of the down projection's epilogue (same result)."""
+    instead of the down projection's epilogue (same result bit for bit)."""
     T, d = x.shape
     E, _, f = w_gate.shape
     sc = _scales(scales)

@@ -24,10 +24,6 @@ constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swiz
 constexpr int X_BYTES = BM * BK * 2;    // 16 KB
 constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16, 128-B swizzle
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
-// The producers prefetch the weight boxes of the K block this many stages
-// ahead of the one they load into L2, so that the weight stream's DRAM latency
-// is covered by L2 rather than by the shared-memory ring alone.
-constexpr int kL2PrefetchStages = 8;
 
 enum { GATEUP = 0, DOWN = 1 };
 
@@ -361,6 +357,83 @@ __device__ __forceinline__ void combine_arrive(const Params& p, const Tile& t, i
     const int src = __ffs(m) - 1;
     m &= m - 1;
     combine_columns(p, __shfl_sync(0xffffffffu, tok, src), t.n0, lane);
+  }
+}
+
+// Weight-stream form of the same combine. There an epilogue warp q holds
+// output columns n0 + 32q + lane and n0 + 128 + 32q + lane of every token row of
+// the tile, so the meeting point is per (token, 256-column tile, warp): each
+// warp counts its own 64 columns of a token and the arrival that completes that
+// count (2 * splits pieces) sums them. No warp waits for another.
+__device__ __forceinline__ void ws_combine_token(const Params& p, int tok, int n0, int q, int lane) {
+  const int64_t p0 = p.slot_pos[2 * static_cast<int64_t>(tok)];
+  const int64_t p1 = p.slot_pos[2 * static_cast<int64_t>(tok) + 1];
+  if (kDebugBounds && !(index_ok(p0, p.rows) && index_ok(p1, p.rows))) {
+    if (lane == 0) atomicOr(p.status, kStatusBounds);
+    return;
+  }
+  const float* y = static_cast<const float*>(p.out);
+  const int64_t ca = n0 + 32 * q + lane, cb = ca + 128;
+  float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;  // slot 0 / slot 1, columns ca / cb
+  for (int s = 0; s < p.splits; ++s) {
+    const float* r0 = y + s * p.split_stride + p0 * p.N;
+    const float* r1 = y + s * p.split_stride + p1 * p.N;
+    a0 += __ldcg(r0 + ca);
+    a1 += __ldcg(r0 + cb);
+    b0 += __ldcg(r1 + ca);
+    b1 += __ldcg(r1 + cb);
+  }
+  float oa = a0 + b0, ob = a1 + b1;
+  const int64_t at = static_cast<int64_t>(tok) * p.N;
+  if (p.residual != nullptr) {
+    oa += __bfloat162float(p.residual[at + ca]);
+    ob += __bfloat162float(p.residual[at + cb]);
+  }
+  p.combine_out[at + ca] = __float2bfloat16_rn(oa);
+  p.combine_out[at + cb] = __float2bfloat16_rn(ob);
+  __syncwarp();
+  if (lane == 0) {  // this warp's two 128-byte lines of every piece are dead
+    for (int s = 0; s < p.splits; ++s) {
+      const float* r0 = y + s * p.split_stride + p0 * p.N;
+      const float* r1 = y + s * p.split_stride + p1 * p.N;
+      discard_l2_line(r0 + n0 + 32 * q);
+      discard_l2_line(r0 + n0 + 128 + 32 * q);
+      discard_l2_line(r1 + n0 + 32 * q);
+      discard_l2_line(r1 + n0 + 128 + 32 * q);
+    }
+  }
+}
+
+// Called by a whole weight-stream epilogue warp after its lanes stored their
+// columns of every row of the tile (rows t.row0 .. t.row0 + t.rows - 1).
+__device__ __forceinline__ void ws_combine_arrive(const Params& p, const Tile& t, int q, int lane) {
+  __threadfence();  // every lane's pieces are visible device-wide before any row is counted
+  __syncwarp();
+  const int64_t per_tok = static_cast<int64_t>(p.N / 256) * 4;
+  for (int r0 = 0; r0 < t.rows; r0 += 32) {
+    const int r = r0 + lane;
+    int tok = 0;
+    bool last = false;
+    if (r < t.rows) {
+      tok = p.perm_token[t.row0 + r];
+      bool ok = true;
+      if (kDebugBounds && !index_ok(tok, p.rows / 2)) {
+        atomicOr(p.status, kStatusBounds);
+        ok = false;
+      }
+      if (ok) {
+        const int old = atomic_add_acq_rel_gpu(&p.combine_count[tok * per_tok + (t.n0 / 256) * 4 + q], 1);
+        last = old == 2 * p.splits - 1;
+      }
+    }
+    unsigned m = __ballot_sync(0xffffffffu, last);
+    if (m == 0) continue;
+    __syncwarp();
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      ws_combine_token(p, __shfl_sync(0xffffffffu, tok, src), t.n0, q, lane);
+    }
   }
 }
 

@@ -87,6 +87,13 @@ constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ri
 // tiles that share one weight tile) go to CTAs that became free together, so
 // they read that weight tile from L2 close in time.
 constexpr int kTileQS = 4;
+// int8 weights: the converter warps form kConvGroups groups that take the
+// K-block steps in turn (group g converts steps n with n % kConvGroups == g),
+// so that several steps are converted at once. One step's conversion is a
+// short chain with a long latency (shared-memory loads, the conversion, the
+// stores and the proxy fence before the MMA may read them); with every warp on
+// the same step the rate was one step per that latency.
+constexpr int kConvGroups = 2;
 static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages &&
                   Cfg<true, false, true>::CSTAGES <= kMaxCStages,
               "converted-W ring deeper than its barrier slots");
@@ -133,11 +140,12 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      // int8: freed by the MMA commit (X read) and every converter warp (W8 read)
-      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_WARPS : 1);
+      // int8: freed by the MMA commit (X read) and the converter warps of the
+      // group that converted it (W8 read)
+      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_WARPS / kConvGroups : 1);
     }
     for (int c = 0; c < C::CSTAGES; ++c) {
-      mbar_init(&cfull_bar[c], C::CONVERT_WARPS);
+      mbar_init(&cfull_bar[c], C::CONVERT_WARPS / kConvGroups);
       mbar_init(&cempty_bar[c], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -259,22 +267,6 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
             } else if (!G) {
               tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
               if (TALL) tma_load_2d(xs + X_BYTES, &tm_x, &full_bar[stage], k0, t.row0 + BM);
-            }
-            // L2 prefetch of the weight boxes kL2PrefetchStages K blocks ahead
-            // (at a tile's first block: of all blocks up to there).
-            for (int ka = kb == 0 ? 1 : kL2PrefetchStages; ka <= kL2PrefetchStages; ++ka) {
-              if (kb + ka >= p.kb_per_split) break;
-              const int kp = k0 + ka * BK;
-              if (W8) {
-                tma_prefetch_l2_3d(&tm_w0, t.n0, kp, t.e);
-                if (KIND == GATEUP) tma_prefetch_l2_3d(&tm_w1, t.n0, kp, t.e);
-                else tma_prefetch_l2_3d(&tm_w0, t.n0 + 128, kp, t.e);
-              } else {
-                for (int j = 0; j < 4; ++j) {
-                  const CUtensorMap* m = (KIND == GATEUP && j >= 2) ? &tm_w1 : &tm_w0;
-                  tma_prefetch_l2_3d(m, t.n0 + 64 * (KIND == GATEUP ? (j & 1) : j), kp, t.e);
-                }
-              }
             }
             if (W8) {
               if (KIND == GATEUP) {
@@ -474,6 +466,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
               }
             }
           }
+          if (p.combine_count != nullptr) ws_combine_arrive(p, t, q, lane);
         }
       }
       tc_fence_before();
@@ -488,11 +481,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     // Staging: two int8 boxes [64 K][128 N] (row = 128 B) in TMA slot `stage`.
     // Target: converted slot `cstage`, four fp16 chunks [64 K][64 N] with the
     // 128-B swizzle (16-B unit u of row k stored at unit u ^ (k % 8)).
-    const int ct = threadIdx.x - 256;  // 0 .. CONVERT_THREADS-1
-    int stage = 0;
-    uint32_t phase = 0;
-    int cstage = 0;
-    uint32_t cphase = 0;
+    constexpr int GWARPS = C::CONVERT_WARPS / kConvGroups;  // warps per group
+    constexpr int GTHREADS = 32 * GWARPS;
+    const int grp = (warp - 8) / GWARPS;
+    const int ct = threadIdx.x - 256 - grp * GTHREADS;  // 0 .. GTHREADS-1 within the group
+    int n = 0;  // K-block step of this CTA, counted over all its tiles
     Tile t;
     for (int i = 0;; ++i) {
       const int tile = dyn ? q_take_warp(i) : static_cast<int>(blockIdx.x + i * gridDim.x);
@@ -502,7 +495,13 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
         goto convert_done;
       }
       if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
-      for (int kb = 0; kb < p.kb_per_split; ++kb) {
+      for (int kb = 0; kb < p.kb_per_split; ++kb, ++n) {
+        if (n % kConvGroups != grp) continue;  // another group's step
+        const int stage = n % STAGES;
+        const uint32_t phase = (n / STAGES) & 1;
+        constexpr int CS = C::CSTAGES > 0 ? C::CSTAGES : 1;  // (this branch runs with int8 weights only)
+        const int cstage = n % CS;
+        const uint32_t cphase = (n / CS) & 1;
         if (!warp_wait(&full_bar[stage], phase, abort_flag) || !warp_wait(&cempty_bar[cstage], cphase ^ 1, abort_flag)) {
           atomicOr(p.status, kStatusConvertTimeout);
           *abort_flag = 1;
@@ -512,22 +511,13 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
           const uint8_t* w8 = smem + stage * C::SLOT_BYTES + C::XS_BYTES;
           uint8_t* wc = conv_area + cstage * W_BYTES;
 #pragma unroll
-          for (int it = 0; it < 1024 / C::CONVERT_THREADS; ++it)
-            convert_int8_segment(w8, wc, ct + C::CONVERT_THREADS * it);
+          for (int it = 0; it < 1024 / GTHREADS; ++it) convert_int8_segment(w8, wc, ct + GTHREADS * it);
         }
         fence_proxy_async_smem();  // this thread's converted stores visible to the async proxy
         __syncwarp();              // ... and the whole warp's, before one arrive per warp
         if (lane == 0) {
           mbar_arrive(&empty_bar[stage]);  // staging slot read
           mbar_arrive(&cfull_bar[cstage]);
-        }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if (++cstage == C::CSTAGES) {
-          cstage = 0;
-          cphase ^= 1;
         }
       }
     }
@@ -595,7 +585,7 @@ cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
   p.select = a.select;
   p.sm_count = device_sm_count();
   p.status = a.status;
-  const bool fuse = KIND == DOWN && !WS && a.combine_count != nullptr;
+  const bool fuse = KIND == DOWN && a.combine_count != nullptr;
   p.perm_token = fuse ? a.perm_token : nullptr;
   p.slot_pos = fuse ? a.slot_pos : nullptr;
   p.combine_count = fuse ? a.combine_count : nullptr;

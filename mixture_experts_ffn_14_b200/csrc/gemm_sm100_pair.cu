@@ -228,16 +228,6 @@ __global__ void __launch_bounds__(PairCfg<W8>::THREADS, 1)
           uint8_t* ws = xs + X_BYTES;
           uint8_t* w8 = ws + PW_BYTES;
           const int k0 = (t.kb0 + kb) * BK;
-          // L2 prefetch of this CTA's weight boxes kL2PrefetchStages K blocks
-          // ahead (at a tile's first block: of all blocks up to there).
-          if (!G || lane == 0) {
-            for (int ka = kb == 0 ? 1 : kL2PrefetchStages; ka <= kL2PrefetchStages; ++ka) {
-              if (kb + ka >= p.kb_per_split) break;
-              const int kp = k0 + ka * BK;
-              tma_prefetch_l2_3d(wmap, n, kp, t.e);
-              if (!W8) tma_prefetch_l2_3d(wmap, n + 64, kp, t.e);
-            }
-          }
           if (W8) {
             if (!G || lane == 0) {
               mbar_arrive_expect_tx(&full_bar[stage], X_BYTES + PW8_BYTES);

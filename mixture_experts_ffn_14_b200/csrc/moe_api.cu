@@ -244,9 +244,10 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   L.router_slices = router_slices(T, d, dtype);
   L.status = take(kAlign);
   L.arrivals = take(sizeof(int32_t) * L.nblk);  // right after the status word: one memset clears both
-  // Token tiles: arrival counters of the combine in the down-projection
-  // epilogue, one per (token, 256-column tile); cleared by the same memset.
-  L.combine_count = L.tile_path ? take(sizeof(int32_t) * T * (d / 256)) : o;
+  // Arrival counters of the combine in the down-projection epilogue, cleared
+  // by the same memset: one per (token, 256-column tile) for token tiles, one
+  // per (token, 256-column tile, epilogue warp) for weight-stream tiles.
+  L.combine_count = dtype == MOE_F32 ? o : take(sizeof(int32_t) * T * (d / 256) * (L.weight_stream ? 4 : 1));
   L.idx = take(sizeof(int32_t) * rows);
   L.gates = take(sizeof(float) * rows);
   L.hist = take(sizeof(int32_t) * L.nblk * kE);
@@ -320,10 +321,10 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   void* h = h_ext ? dbg->h : static_cast<void*>(ws + L.h);
   float* y = reinterpret_cast<float*>(ws + L.y);
   const int64_t T = a->T, d = a->d, f = a->f;
-  // Token tiles sum each token's two rows in the down projection's epilogue;
-  // a separate combine kernel runs for the weight-stream and fp32 paths, with
-  // the post-RMSNorm (it needs whole rows), or when asked for.
-  const bool fused_combine = L.tile_path && !o->post_norm_weight && o->separate_combine == 0;
+  // The down projection's epilogue sums each token's rows (token tiles and
+  // weight-stream tiles); a separate combine kernel runs for the fp32 path,
+  // with the post-RMSNorm (it needs whole rows), or when asked for.
+  const bool fused_combine = a->dtype != MOE_F32 && !o->post_norm_weight && o->separate_combine == 0;
   int32_t* combine_count = reinterpret_cast<int32_t*>(ws + L.combine_count);
 
 #define MOE_TRY(call)                                  \

@@ -257,6 +257,9 @@ def test_bitwise_determinism_and_streams():
 
 
 @pytest.mark.parametrize("T,path,int8,splits,residual,skew", [
+    (64, moe.MOE_PATH_AUTO, False, 0, False, False),           # weight-stream, split-K
+    (100, moe.MOE_PATH_WEIGHT_STREAM, True, 3, True, False),
+    (200, moe.MOE_PATH_WEIGHT_STREAM, False, 1, True, True),
     (300, moe.MOE_PATH_TOKEN_TILE, False, 1, False, False),
     (300, moe.MOE_PATH_TOKEN_TILE_SINGLE, False, 3, True, False),
     (1000, moe.MOE_PATH_AUTO, False, 0, False, False),
@@ -265,10 +268,11 @@ def test_bitwise_determinism_and_streams():
     (517, moe.MOE_PATH_TOKEN_TILE_SINGLE, True, 1, False, True),
 ])
 def test_fused_combine_matches_combine_kernel_bitwise(T, path, int8, splits, residual, skew):
-    # Token tiles sum each token's rows in the down projection's epilogue
-    # (whichever tile finishes last, in a fixed order); the separate combine
-    # kernel sums the same pieces in the same order: outputs equal bit for bit,
-    # also with split-K pieces, the residual add, int8 tiles and skewed loads.
+    # The down projection's epilogue sums each token's rows (whichever tile
+    # finishes last, in a fixed order; token tiles and weight-stream tiles);
+    # the separate combine kernel sums the same pieces in the same order:
+    # outputs equal bit for bit, also with split-K pieces, the residual add,
+    # int8 tiles and skewed loads.
     inp = small_bf16(T, seed=110 + T, int8=int8, skew=skew)
     kw = {}
     if residual:

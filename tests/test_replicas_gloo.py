@@ -49,10 +49,9 @@ def test_two_replicas_max_time_and_summed_work():
 def test_launch_count_rule():
     from mixture_experts_ffn_14_b200 import workloads as W
 
-    # Token tiles combine in the down projection's epilogue (no combine kernel);
-    # the weight-stream path (decode) keeps one.
+    # The down projection's epilogue sums each token's rows: no combine kernel.
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "auto") == 6
-    assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 5
+    assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 4
     assert bench.launches_per_step(W.WORKLOADS["int8"], "auto") == 4
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "token_tile") == 4
     assert bench.launches_per_step(W.WORKLOADS["skewed"], "auto") == 6
