@@ -87,13 +87,13 @@ constexpr int kMaxCStages = 4;  // barrier slots reserved for the converted-W ri
 // tiles that share one weight tile) go to CTAs that became free together, so
 // they read that weight tile from L2 close in time.
 constexpr int kTileQS = 4;
-// int8 weights: the converter warps form kConvGroups groups that take the
-// K-block steps in turn (group g converts steps n with n % kConvGroups == g),
-// so that several steps are converted at once. One step's conversion is a
-// short chain with a long latency (shared-memory loads, the conversion, the
-// stores and the proxy fence before the MMA may read them); with every warp on
-// the same step the rate was one step per that latency.
-constexpr int kConvGroups = 2;
+// int8 weights: the converter warps form conv_groups(WS) groups that take the
+// K-block steps in turn (group g converts steps n with n % groups == g), so
+// that several steps are converted at once. Measured (two alternating runs
+// each): weight-stream (decode, T = 64) 1.458 -> 1.420 ms with two groups;
+// 256-row token tiles slower with two (T = 1024 2.91 -> 2.99 ms, T = 4096 8.94
+// -> 9.16 ms), so they keep one group of eight warps on each step.
+__host__ __device__ constexpr int conv_groups(bool ws) { return ws ? 2 : 1; }
 static_assert(Cfg<true>::CSTAGES <= kMaxCStages && Cfg<true, true>::CSTAGES <= kMaxCStages &&
                   Cfg<true, false, true>::CSTAGES <= kMaxCStages,
               "converted-W ring deeper than its barrier slots");
@@ -142,10 +142,10 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       mbar_init(&full_bar[s], 1);
       // int8: freed by the MMA commit (X read) and the converter warps of the
       // group that converted it (W8 read)
-      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_WARPS / kConvGroups : 1);
+      mbar_init(&empty_bar[s], W8 ? 1 + C::CONVERT_WARPS / conv_groups(WS) : 1);
     }
     for (int c = 0; c < C::CSTAGES; ++c) {
-      mbar_init(&cfull_bar[c], C::CONVERT_WARPS / kConvGroups);
+      mbar_init(&cfull_bar[c], C::CONVERT_WARPS / conv_groups(WS));
       mbar_init(&cempty_bar[c], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -481,7 +481,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     // Staging: two int8 boxes [64 K][128 N] (row = 128 B) in TMA slot `stage`.
     // Target: converted slot `cstage`, four fp16 chunks [64 K][64 N] with the
     // 128-B swizzle (16-B unit u of row k stored at unit u ^ (k % 8)).
-    constexpr int GWARPS = C::CONVERT_WARPS / kConvGroups;  // warps per group
+    constexpr int GROUPS = conv_groups(WS);
+    constexpr int GWARPS = C::CONVERT_WARPS / GROUPS;  // warps per group
     constexpr int GTHREADS = 32 * GWARPS;
     const int grp = (warp - 8) / GWARPS;
     const int ct = threadIdx.x - 256 - grp * GTHREADS;  // 0 .. GTHREADS-1 within the group
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       }
       if (tile < 0 || !decode_tile(*sched, p, tile, TROWS, t)) break;
       for (int kb = 0; kb < p.kb_per_split; ++kb, ++n) {
-        if (n % kConvGroups != grp) continue;  // another group's step
+        if (n % GROUPS != grp) continue;  // another group's step
         const int stage = n % STAGES;
         const uint32_t phase = (n / STAGES) & 1;
         constexpr int CS = C::CSTAGES > 0 ? C::CSTAGES : 1;  // (this branch runs with int8 weights only)
