@@ -516,7 +516,9 @@ def recorded_traffic(wl):
     import re
 
     records = {("prefill", 4096, 6144, 32768): "gemm_traffic_prefill_T4096.md",
-               ("decode", 64, 6144, 32768): "gemm_traffic_decode_T64.md"}
+               ("decode", 64, 6144, 32768): "gemm_traffic_decode_T64.md",
+               ("int8", 1024, 6144, 32768): "gemm_traffic_int8_T1024.md",
+               ("skewed", 16384, 6144, 32768): "gemm_traffic_skewed_T16384.md"}
     name = records.get((wl.name, wl.T, wl.d, wl.f))
     path = os.path.join(ROOT, "profiles", name) if name else None
     if not path or not os.path.exists(path):

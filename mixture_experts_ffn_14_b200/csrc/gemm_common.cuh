@@ -13,6 +13,7 @@
 
 #include "moe_internal.cuh"
 #include "sm100.cuh"
+#include "tile_order.cuh"
 
 namespace moe {
 namespace tc {
@@ -24,6 +25,8 @@ constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-B swiz
 constexpr int X_BYTES = BM * BK * 2;    // 16 KB
 constexpr int WCHUNK = BK * 64 * 2;     // 8 KB: [64 K x 64 N] bf16, 128-B swizzle
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no wait is unbounded
+constexpr long long kL2GroupBytes = 64ll << 20;     // activation rows of one row-tile group
+constexpr long long kL2UngroupedBytes = 96ll << 20; // an expert's rows above this are grouped
 
 enum { GATEUP = 0, DOWN = 1 };
 
@@ -44,7 +47,9 @@ struct Params {
   int32_t act;           // moe_activation_t of the gate branch
   int32_t select;        // kRunAlways, or run only if the pair / single form is preferred
   int32_t sm_count;      // SMs of the device (same value for both token-tile kernels)
-  int32_t* tile_counter; // CTA-pair kernel, bf16 weights: tiles handed out in order (zero on entry)
+  int32_t* tile_counter; // tiles handed out in order (zero on entry), or nullptr (static order)
+  int32_t group_rows;    // row tiles per L2 group (tile_order.cuh) ...
+  int32_t group_limit;   // ... for experts with more row tiles than this
   uint32_t* status;
   // DOWN token tiles with the combine in the epilogue (combine_count != nullptr)
   const int32_t* perm_token;
@@ -131,12 +136,8 @@ __device__ __forceinline__ bool decode_tile(const SharedSched& s, const Params& 
   if (tile >= s.pre[kE]) return false;
   int e = 0;
   while (tile >= s.pre[e + 1]) ++e;
-  const int local = tile - s.pre[e];
-  const int nt_count = p.N / p.ntile;
-  const int mt = local % s.mt[e];
-  const int rest = local / s.mt[e];
-  const int nt = rest % nt_count;
-  const int ks = rest / nt_count;
+  int mt, nt, ks;
+  tile_coords(tile - s.pre[e], s.mt[e], p.N / p.ntile, group_for(s.mt[e], p.group_rows, p.group_limit), mt, nt, ks);
   t.e = e;
   t.row0 = s.off[e] + mt * tile_rows;
   t.rows = min(tile_rows, s.cnt[e] - mt * tile_rows);

@@ -488,6 +488,10 @@ cudaError_t launch_pair(const TcGemmArgs& a, cudaStream_t stream) {
   p.splits = KIND == DOWN ? a.splits : 1;
   p.kb_per_split = a.K / BK / p.splits;
   p.ntile = KIND == GATEUP ? 128 : 256;
+  // L2 groups of row tiles (tile_order.cuh): experts whose activation rows
+  // (this K split) exceed 96 MB go in groups of 64 MB.
+  p.group_rows = row_group_size(PAIR_ROWS, int64_t(p.kb_per_split) * BK, kL2GroupBytes);
+  p.group_limit = row_group_size(PAIR_ROWS, int64_t(p.kb_per_split) * BK, kL2UngroupedBytes);
   p.act = a.act;
   p.select = a.select;
   p.sm_count = device_sm_count();

@@ -1,6 +1,7 @@
-"""The index predicates of the MOE_DEBUG_BOUNDS build, compiled for the host
-and run with in-range and out-of-range indices (no GPU); and the debug build
-of the library loads and reports its flag."""
+"""Host-compiled checks of device logic (no GPU): the index predicates of the
+MOE_DEBUG_BOUNDS build with in-range and out-of-range indices, and the
+token-tile order of the expert GEMMs; and the debug build of the library loads
+and reports its flag."""
 
 import os
 import shutil
@@ -23,6 +24,18 @@ def test_bounds_predicates_on_host(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "bounds predicates ok" in r.stdout
+
+
+def test_tile_order_is_a_grouped_bijection(tmp_path):
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.fail("no host C++ compiler")
+    exe = tmp_path / "tile_order_check"
+    subprocess.run([cxx, "-std=c++17", "-O2", "-Wall", "-Werror", "-I", CSRC,
+                    os.path.join(ROOT, "tests", "tile_order_host_check.cpp"), "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr
+    assert "tile order ok" in r.stdout
 
 
 def test_debug_build_loads_and_reports_its_flag():

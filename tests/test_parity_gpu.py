@@ -403,6 +403,21 @@ def test_int8_tall_tiles_both_halves(T, skew):
     full_check(inp, g)
 
 
+@pytest.mark.parametrize("path", [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE])
+def test_grouped_tile_order_for_large_experts(path):
+    # An expert whose intermediate rows exceed the L2 budget (here 2000 rows x
+    # f = 32768 for the down projection: 8 pair or 16 single-CTA row tiles of
+    # 16 / 8 MB) has its row tiles taken in groups; every token still routes to
+    # experts 0 and 1, and the outputs match the oracle.
+    w = W.Workload("grouped", 2000, 256, 32768, dtype="bf16", seed=140)
+    inp = W.make_torch(w, DEV)
+    inp["router_bias"] = torch.tensor([40.0, 30.0, 0, 0, 0, 0, 0, 0], device=DEV)
+    gpu = run_gpu(inp, path=path, down_splits=1, want_h=False)
+    assert list(gpu["counts"][:2]) == [2000, 2000]
+    rng = np.random.default_rng(7)
+    full_check(inp, gpu, tokens=np.sort(rng.choice(2000, size=48, replace=False)), check_h=False)
+
+
 def _status_after(inp, x, path=moe.MOE_PATH_AUTO):
     T, d = x.shape
     f = inp["w_gate"].shape[2]
