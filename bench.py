@@ -342,14 +342,16 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 
 
 def launches_per_step(wl, path):
-    """Kernels of ours per step: router, dispatch and two GEMMs (the down
-    projection's epilogue sums each token's rows, so no combine kernel runs);
-    with the automatic token-tile choice on bf16 weights each GEMM launches both
-    forms (the one not chosen returns at once); above 1024 router blocks
-    (T > 32768) a histogram scan runs before the dispatch."""
+    """Kernels of ours per step: router, dispatch (one cluster launch for both
+    at T <= 128) and two GEMMs (the down projection's epilogue sums each
+    token's rows, so no combine kernel runs); with the automatic token-tile
+    choice on bf16 weights each GEMM launches both forms (the one not chosen
+    returns at once); above 1024 router blocks (T > 32768) a histogram scan
+    runs before the dispatch."""
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
-    return 4 + (2 if both else 0) + (1 if scan else 0)
+    route = 1 if wl.T <= 128 else 2
+    return route + 2 + (2 if both else 0) + (1 if scan else 0)
 
 
 # ---------------------------------------------------------------- main --

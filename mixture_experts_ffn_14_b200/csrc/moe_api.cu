@@ -339,11 +339,19 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   // zero (contiguous regions, up to the next one).
   MOE_TRY(cudaMemsetAsync(status, 0, L.idx - L.status, stream));
   MOE_TRY(mark(0));
-  MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, L.router_slices,
-                        logits_part, arrivals, idx, gates, hist, stream));
-  MOE_TRY(mark(1));
-  MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, hist_pre, counts, offsets, perm_token,
-                          perm_slot, slot_pos, gate_perm, xp, status, stream));
+  if (small_route_dispatch(T, xp)) {
+    // Decode-sized batches: router and dispatch in one cluster launch.
+    MOE_TRY(launch_route_dispatch_small(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, idx,
+                                        gates, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm, xp,
+                                        status, stream));
+    MOE_TRY(mark(1));
+  } else {
+    MOE_TRY(launch_router(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, L.router_slices,
+                          logits_part, arrivals, idx, gates, hist, stream));
+    MOE_TRY(mark(1));
+    MOE_TRY(launch_dispatch(a->dtype, a->x, T, d, L.nblk, idx, gates, hist, hist_pre, counts, offsets,
+                            perm_token, perm_slot, slot_pos, gate_perm, xp, status, stream));
+  }
   MOE_TRY(mark(2));
   if (a->dtype == MOE_F32) {
     MOE_TRY(launch_f32_gateup(static_cast<const float*>(xp), static_cast<const float*>(a->w_gate),
@@ -692,6 +700,12 @@ moe_status_t moe_route_dispatch(const void* x, const float* w_router, const floa
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   if (cudaMemsetAsync(status, 0, L.logits_part ? L.logits_part - L.status : L.hist - L.status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
+  if (small_route_dispatch(T, r->xp))
+    return launch_route_dispatch_small(dtype, x, w_router, router_bias, T, d, renormalize, r->idx, r->gates,
+                                       r->counts, r->offsets, r->perm_token, r->perm_slot, r->slot_pos,
+                                       r->gate_perm, r->xp, status, s) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
   if (launch_router(dtype, x, w_router, router_bias, T, d, renormalize, L.slices,
                     L.slices > 1 ? reinterpret_cast<float*>(ws + L.logits_part) : nullptr,
                     reinterpret_cast<int32_t*>(ws + L.arrivals), r->idx, r->gates, hist, s) != cudaSuccess)

@@ -18,6 +18,7 @@
 #include <cstdint>
 
 #include "moe_internal.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
@@ -458,6 +459,203 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
   if (F16 && f16_bad) atomicOr(status, kStatusFp16Range);
 }
 
+// ---- small batches: router and dispatch in one cluster launch -------------
+// For T <= kSmallMaxT (decode) the two stages above cost more in launches and
+// global round trips (partial logits, an arrival counter, a second kernel)
+// than in work. Here one cluster of kSmallCTAs CTAs does both:
+//   1. CTA c forms the partial logits of every token over its slice of the
+//      hidden dimension (d / kSmallCTAs elements; the slice's router weights
+//      staged through shared memory as in the router kernel) and keeps them in
+//      its shared memory;
+//   2. cluster barrier; CTA 0 sums each token's partials in slice order
+//      (reading the other CTAs' shared memory), finishes the routing exactly
+//      as the router kernel does (same top-2, softmax and gate arithmetic) and
+//      computes counts, offsets and the stable (expert, token) permutation;
+//   3. cluster barrier; every CTA copies its share of the 2T permuted rows of
+//      x (converted to fp16 for int8 weights), reading the positions from CTA 0;
+//   4. cluster barrier, so CTA 0's shared memory outlives those reads.
+constexpr int kSmallCTAs = 8;
+constexpr int kSmallMaxT = 128;
+constexpr int kSmallThreads = 256;
+
+template <typename TX, bool F16 = false>
+__global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThreads)
+    moe_route_dispatch_small_kernel(const TX* __restrict__ x, const float* __restrict__ wr,
+                                    const float* __restrict__ bias, int64_t T, int64_t d, int32_t renormalize,
+                                    int32_t* __restrict__ idx, float* __restrict__ gates,
+                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                    int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
+                                    int32_t* __restrict__ slot_pos, float* __restrict__ gate_perm,
+                                    TX* __restrict__ xp, uint32_t* __restrict__ status) {
+  using namespace moe::sm100;
+  constexpr int V = Vec<TX>::N;
+  __shared__ float part[kSmallMaxT][kE];  // this CTA's partial logits
+  __shared__ int sel[kSmallMaxT][2];      // CTA 0: chosen experts
+  __shared__ float sgate[kSmallMaxT][2];  // CTA 0: their gates
+  __shared__ int pos[kSmallMaxT][2];      // CTA 0: permuted row of each (token, slot)
+  __shared__ int cnt[kE];
+  __shared__ float4 wsm[(kWrRows * kE + (kWrRows / 4) * 4) / 4];
+  const uint32_t rank = cluster_ctarank();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  constexpr int kWarps = kSmallThreads / 32;
+  if (threadIdx.x < kE) cnt[threadIdx.x] = 0;
+
+  // 1. Partial logits over this CTA's slice, kTokPerWarp tokens per warp pass.
+  const int64_t len = d / kSmallCTAs;
+  const int64_t c_begin = static_cast<int64_t>(rank) * len;
+  for (int64_t tb = static_cast<int64_t>(warp) * kTokPerWarp; tb < kSmallMaxT; tb += kWarps * kTokPerWarp) {
+    // every warp runs the same number of passes (the __syncthreads below)
+    const TX* rows[kTokPerWarp];
+#pragma unroll
+    for (int j = 0; j < kTokPerWarp; ++j) rows[j] = x + min(tb + j, T - 1) * d;  // clamped: always in bounds
+    float acc[kTokPerWarp][kE];
+#pragma unroll
+    for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+      for (int e = 0; e < kE; ++e) acc[j][e] = 0.0f;
+    for (int64_t cc = c_begin; cc < c_begin + len; cc += kWrRows) {
+      const int rows_here = static_cast<int>(min(static_cast<int64_t>(kWrRows), c_begin + len - cc));
+      __syncthreads();
+      for (int q = threadIdx.x; q < rows_here * 2; q += blockDim.x) {
+        const int r = q >> 1;
+        wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] =
+            *reinterpret_cast<const float4*>(wr + (cc + r) * kE + (q & 1) * 4);
+      }
+      __syncthreads();
+      if (tb < T) {
+        for (int r0 = lane * V; r0 < rows_here; r0 += 32 * V) {
+          float xv[kTokPerWarp][V];
+#pragma unroll
+          for (int j = 0; j < kTokPerWarp; ++j) Vec<TX>::load(rows[j] + cc + r0, xv[j]);
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            const int r = r0 + i;
+            const float4 a = wsm[(r * kE + (r / V) * 4) / 4];
+            const float4 b = wsm[(r * kE + (r / V) * 4) / 4 + 1];
+            const float w[kE] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+              for (int e = 0; e < kE; ++e) acc[j][e] = fmaf(xv[j][i], w[e], acc[j][e]);
+          }
+        }
+      }
+    }
+    if (tb < T) {
+#pragma unroll
+      for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+        for (int e = 0; e < kE; ++e) acc[j][e] = warp_sum(acc[j][e]);
+      if (lane < kTokPerWarp) {
+#pragma unroll
+        for (int j = 0; j < kTokPerWarp; ++j)
+          if (lane == j)
+#pragma unroll
+            for (int e = 0; e < kE; ++e) part[tb + j][e] = acc[j][e];
+      }
+    }
+  }
+  cluster_sync();
+
+  // 2. CTA 0: routing and the permutation.
+  if (rank == 0) {
+    const int t = threadIdx.x;
+    if (t < T) {
+      float l[kE], sum[kE];
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        l[e] = bias ? bias[e] : 0.0f;
+        sum[e] = 0.0f;
+      }
+      for (uint32_t c = 0; c < kSmallCTAs; ++c) {
+        const uint32_t at = mapa_shared(&part[t][0], c);
+#pragma unroll
+        for (int e = 0; e < kE; ++e) sum[e] += ld_shared_cluster_f32(at + 4 * e);
+      }
+#pragma unroll
+      for (int e = 0; e < kE; ++e) l[e] += sum[e];
+      finalize_token(l, t, renormalize, idx, gates, cnt);
+      // finalize_token wrote idx / gates to global memory; keep this thread's copy
+      sel[t][0] = idx[2 * t];
+      sel[t][1] = idx[2 * t + 1];
+      sgate[t][0] = gates[2 * t];
+      sgate[t][1] = gates[2 * t + 1];
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int base[kE];
+      int off = 0;
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        base[e] = off;
+        off += cnt[e];
+      }
+      if (lane < kE) {
+        counts[lane] = cnt[lane];
+        offsets[lane] = base[lane];
+      }
+      if (lane == 0) offsets[kE] = off;
+      const unsigned lt = (1u << lane) - 1u;
+      for (int t0 = 0; t0 < T; t0 += 32) {
+        const int t = t0 + lane;
+        const bool valid = t < T;
+        const int a = valid ? sel[t][0] : -1;
+        const int b = valid ? sel[t][1] : -1;
+        int pa = -1, pb = -1;
+#pragma unroll
+        for (int e = 0; e < kE; ++e) {
+          const unsigned m = __ballot_sync(0xffffffffu, a == e || b == e);
+          const int r = base[e] + __popc(m & lt);
+          if (a == e) pa = r;
+          if (b == e) pb = r;
+          base[e] += __popc(m);
+        }
+        if (valid) {
+          if (kDebugBounds && !(index_ok(pa, 2 * T) && index_ok(pb, 2 * T))) {
+            atomicOr(status, kStatusBounds);
+            pa = pb = -1;
+          } else {
+            perm_token[pa] = t;
+            perm_slot[pa] = 0;
+            perm_token[pb] = t;
+            perm_slot[pb] = 1;
+            slot_pos[2 * t] = pa;
+            slot_pos[2 * t + 1] = pb;
+            gate_perm[pa] = sgate[t][0];
+            gate_perm[pb] = sgate[t][1];
+          }
+          pos[t][0] = pa;
+          pos[t][1] = pb;
+        }
+      }
+    }
+  }
+  cluster_sync();
+
+  // 3. The permuted copy of x, rows spread over the cluster's warps.
+  const int64_t vec_per_row = d * static_cast<int64_t>(sizeof(TX)) / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+  uint4* dst = reinterpret_cast<uint4*>(xp);
+  uint32_t f16_bad = 0;
+  for (int64_t r = static_cast<int64_t>(rank) * kWarps + warp; r < 2 * T; r += kSmallCTAs * kWarps) {
+    const int64_t t = r >> 1;
+    const int p = ld_shared_cluster_s32(mapa_shared(&pos[t][r & 1], 0));
+    if (p < 0) continue;
+    for (int64_t c = lane; c < vec_per_row; c += 32) {
+      const uint4 v = src[t * vec_per_row + c];
+      if (F16) {
+        const uint4 h = bf16x8_to_f16x8(v);
+        f16_bad |= f16x8_nonfinite(h);
+        dst[static_cast<int64_t>(p) * vec_per_row + c] = h;
+      } else {
+        dst[static_cast<int64_t>(p) * vec_per_row + c] = v;
+      }
+    }
+  }
+  if (F16 && f16_bad) atomicOr(status, kStatusFp16Range);
+  cluster_sync();  // CTA 0's shared memory stays until every CTA has read it
+}
+
 template <typename TO>
 __device__ __forceinline__ void store4(TO* p, float4 v);
 
@@ -656,6 +854,29 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
     moe_dispatch_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), T, d, nblk, idx, gates, hist, counts, offsets, perm_token,
         perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), pre, tot, status);
+  return cudaGetLastError();
+}
+
+bool small_route_dispatch(int64_t T, const void* xp) { return T > 0 && T <= kSmallMaxT && xp != nullptr; }
+
+cudaError_t launch_route_dispatch_small(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias,
+                                        int64_t T, int64_t d, int32_t renormalize, int32_t* idx, float* gates,
+                                        int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
+                                        int32_t* slot_pos, float* gate_perm, void* xp, uint32_t* status,
+                                        cudaStream_t s) {
+  const dim3 grid(kSmallCTAs), block(kSmallThreads);
+  if (dtype == MOE_F32)
+    moe_route_dispatch_small_kernel<float><<<grid, block, 0, s>>>(
+        static_cast<const float*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets, perm_token,
+        perm_slot, slot_pos, gate_perm, static_cast<float*>(xp), status);
+  else if (dtype == MOE_BF16_INT8W)
+    moe_route_dispatch_small_kernel<__nv_bfloat16, true><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets,
+        perm_token, perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), status);
+  else
+    moe_route_dispatch_small_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets,
+        perm_token, perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), status);
   return cudaGetLastError();
 }
 

@@ -130,3 +130,28 @@ def test_gather_rows_and_combine_entry_points():
     out = comp.combine(routed, y)
     ref = (y[perm[:, 0].long()] + y[perm[:, 1].long()]).to(torch.bfloat16)
     assert torch.equal(out, ref)
+
+
+def test_expert_parallel_over_nccl_single_rank():
+    # The multi-GPU code path itself (DistExchange over a torch.distributed NCCL
+    # group, LibraryCompute through the C ABI) with one rank: every exchange is
+    # a copy to itself, and the result must equal the single-GPU forward bit for
+    # bit with the same kernel form and split-K.
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, device_id=torch.device(DEV))
+    try:
+        full, xs = _inputs(1, "bf16", seed=300)
+        comp = _local_compute(full, 0, 1)
+        out = EP.ep_forward(xs[0], comp, EP.DistExchange())
+        torch.cuda.synchronize()
+        assert torch.equal(out, _single_gpu(full, xs[0]))
+    finally:
+        dist.destroy_process_group()

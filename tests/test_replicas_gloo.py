@@ -51,7 +51,7 @@ def test_launch_count_rule():
 
     # The down projection's epilogue sums each token's rows: no combine kernel.
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "auto") == 6
-    assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 4
+    assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 3   # router + dispatch in one launch
     assert bench.launches_per_step(W.WORKLOADS["int8"], "auto") == 4
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "token_tile") == 4
     assert bench.launches_per_step(W.WORKLOADS["skewed"], "auto") == 6
