@@ -339,7 +339,7 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
   // zero (contiguous regions, up to the next one).
   MOE_TRY(cudaMemsetAsync(status, 0, L.idx - L.status, stream));
   MOE_TRY(mark(0));
-  if (small_route_dispatch(T, xp)) {
+  if (small_route_dispatch(T, d, xp)) {
     // Decode-sized batches: router and dispatch in one cluster launch.
     MOE_TRY(launch_route_dispatch_small(a->dtype, a->x, a->w_router, o->router_bias, T, d, o->renormalize, idx,
                                         gates, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm, xp,
@@ -700,7 +700,7 @@ moe_status_t moe_route_dispatch(const void* x, const float* w_router, const floa
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   if (cudaMemsetAsync(status, 0, L.logits_part ? L.logits_part - L.status : L.hist - L.status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (small_route_dispatch(T, r->xp))
+  if (small_route_dispatch(T, d, r->xp))
     return launch_route_dispatch_small(dtype, x, w_router, router_bias, T, d, renormalize, r->idx, r->gates,
                                        r->counts, r->offsets, r->perm_token, r->perm_slot, r->slot_pos,
                                        r->gate_perm, r->xp, status, s) == cudaSuccess

@@ -73,10 +73,11 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
                             int32_t* slot_pos, float* gate_perm, void* xp, uint32_t* status,
                             cudaStream_t s);  // xp == nullptr: no row copy
 
-// Small batches (1 <= T <= 128, with the permuted copy): router and dispatch
-// in one launch of an 8-CTA cluster; same outputs as the two launches above
-// (idx, gates, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm, xp).
-bool small_route_dispatch(int64_t T, const void* xp);
+// Small batches (1 <= T <= 128, d <= 65536, with the permuted copy, and a
+// device on which a 16-CTA cluster fits): router and dispatch in one cluster
+// launch; same outputs as the two launches above (idx, gates, counts, offsets,
+// perm_token, perm_slot, slot_pos, gate_perm, xp).
+bool small_route_dispatch(int64_t T, int64_t d, const void* xp);
 cudaError_t launch_route_dispatch_small(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias,
                                         int64_t T, int64_t d, int32_t renormalize, int32_t* idx, float* gates,
                                         int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,

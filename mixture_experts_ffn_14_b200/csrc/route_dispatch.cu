@@ -33,6 +33,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// The warp sums of 32 values at once, lane L receiving the sum of value L
+// (v[j][e], L = j * kE + e): at each xor step a lane keeps the half of its
+// values that its side of the pairing owns and adds the partner's copy of them,
+// 31 shuffles instead of 5 per value. The pairings are warp_sum's, so every sum
+// has the same bits as warp_sum of that value.
+__device__ __forceinline__ float warp_reduce_scatter(const float (&v)[kTokPerWarp][kE], int lane) {
+  static_assert(kTokPerWarp * kE == 32, "32 values");
+  float a[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a[i] = v[i / kE][i % kE];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? a[i] : a[i + off];
+      const float keep = upper ? a[i + off] : a[i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return a[0];
+}
+
 __device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -45,17 +68,17 @@ struct Vec;  // 16-byte vector of activations
 template <>
 struct Vec<float> {
   static constexpr int N = 4;
-  __device__ static void load(const float* p, float (&v)[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  __device__ static void unpack(const uint4 a, float (&v)[4]) {
+    v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+    v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
   }
+  __device__ static void load(const float* p, float (&v)[4]) { unpack(*reinterpret_cast<const uint4*>(p), v); }
 };
 
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int N = 8;
-  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 a = *reinterpret_cast<const uint4*>(p);
+  __device__ static void unpack(const uint4 a, float (&v)[8]) {
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -63,12 +86,19 @@ struct Vec<__nv_bfloat16> {
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
+  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    unpack(*reinterpret_cast<const uint4*>(p), v);
+  }
+};
+
+struct Top2 {
+  int e0, e1;
+  float g0, g1;
 };
 
 // Top-2 of the 8 logits (strict comparisons keep the lower index on ties),
-// softmax in fp32 and the gates (optionally renormalised), for token t.
-__device__ __forceinline__ void finalize_token(const float (&l)[kE], int64_t t, int32_t renormalize,
-                                               int32_t* __restrict__ idx, float* __restrict__ gates, int* cnt) {
+// softmax in fp32 and the gates (optionally renormalised).
+__device__ __forceinline__ Top2 route_token(const float (&l)[kE], int32_t renormalize) {
   int e0 = 0;
   float m = l[0];
 #pragma unroll
@@ -88,18 +118,23 @@ __device__ __forceinline__ void finalize_token(const float (&l)[kE], int64_t t, 
   float s = 0.0f;
 #pragma unroll
   for (int e = 0; e < kE; ++e) s += expf(l[e] - m);
-  idx[2 * t] = e0;
-  idx[2 * t + 1] = e1;
   const float p1 = expf(m1 - m);
-  if (renormalize) {  // Mixtral: the two probabilities divided by their sum
-    gates[2 * t] = 1.0f / (1.0f + p1);
-    gates[2 * t + 1] = p1 / (1.0f + p1);
-  } else {
-    gates[2 * t] = 1.0f / s;
-    gates[2 * t + 1] = p1 / s;
-  }
-  atomicAdd(&cnt[e0], 1);
-  atomicAdd(&cnt[e1], 1);
+  if (renormalize)  // Mixtral: the two probabilities divided by their sum
+    return Top2{e0, e1, 1.0f / (1.0f + p1), p1 / (1.0f + p1)};
+  return Top2{e0, e1, 1.0f / s, p1 / s};
+}
+
+// route_token for token t: idx / gates stored, the block's expert counts raised.
+__device__ __forceinline__ Top2 finalize_token(const float (&l)[kE], int64_t t, int32_t renormalize,
+                                               int32_t* __restrict__ idx, float* __restrict__ gates, int* cnt) {
+  const Top2 r = route_token(l, renormalize);
+  idx[2 * t] = r.e0;
+  idx[2 * t + 1] = r.e1;
+  gates[2 * t] = r.g0;
+  gates[2 * t + 1] = r.g1;
+  atomicAdd(&cnt[r.e0], 1);
+  atomicAdd(&cnt[r.e1], 1);
+  return r;
 }
 
 // Grid (token blocks of 32, d slices). One warp = 4 tokens; lanes split the CTA's
@@ -143,9 +178,20 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(
   for (int64_t cc = c_begin; cc < c_begin + len; cc += kWrRows) {
     const int rows_here = static_cast<int>(min(static_cast<int64_t>(kWrRows), c_begin + len - cc));
     __syncthreads();
-    for (int q = threadIdx.x; q < rows_here * 2; q += blockDim.x) {
-      const int r = q >> 1;
-      wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] = *reinterpret_cast<const float4*>(wr + (cc + r) * kE + (q & 1) * 4);
+    constexpr int kIt = 4;  // loads issued together before their stores
+    for (int q0 = threadIdx.x; q0 < rows_here * 2; q0 += kIt * kRouterThreads) {
+      float4 wv[kIt];
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int q = q0 + k * kRouterThreads;
+        if (q < rows_here * 2) wv[k] = *reinterpret_cast<const float4*>(wr + (cc + (q >> 1)) * kE + (q & 1) * 4);
+      }
+#pragma unroll
+      for (int k = 0; k < kIt; ++k) {
+        const int q = q0 + k * kRouterThreads;
+        const int r = q >> 1;
+        if (q < rows_here * 2) wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] = wv[k];
+      }
     }
     __syncthreads();
 #pragma unroll 2
@@ -166,30 +212,19 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(
       }
     }
   }
-#pragma unroll
-  for (int j = 0; j < kTokPerWarp; ++j)
-#pragma unroll
-    for (int e = 0; e < kE; ++e) acc[j][e] = warp_sum(acc[j][e]);
+  // lane L: the warp's sum for token t0 + L / 8, expert L % 8
+  const float sum_l = warp_reduce_scatter(acc, lane);
 
   if (slices == 1) {
 #pragma unroll
     for (int j = 0; j < kTokPerWarp; ++j) {
-      if (lane == j && t0 + j < T) {
-        float l[kE];
+      float l[kE];
 #pragma unroll
-        for (int e = 0; e < kE; ++e) l[e] = acc[j][e] + (bias ? bias[e] : 0.0f);
-        finalize_token(l, t0 + j, renormalize, idx, gates, cnt);
-      }
+      for (int e = 0; e < kE; ++e) l[e] = __shfl_sync(0xffffffffu, sum_l, j * kE + e) + (bias ? bias[e] : 0.0f);
+      if (lane == j && t0 + j < T) finalize_token(l, t0 + j, renormalize, idx, gates, cnt);
     }
   } else {
-#pragma unroll
-    for (int j = 0; j < kTokPerWarp; ++j) {
-      if (lane == j && t0 + j < T) {
-        float* dst = partial + (static_cast<int64_t>(blockIdx.y) * T + t0 + j) * kE;
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
-      }
-    }
+    if (t0 + lane / kE < T) partial[(static_cast<int64_t>(blockIdx.y) * T + t0 + lane / kE) * kE + lane % kE] = sum_l;
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) last = atomicAdd(&arrivals[blk], 1) == slices - 1;
@@ -471,15 +506,27 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(
 //      (reading the other CTAs' shared memory), finishes the routing exactly
 //      as the router kernel does (same top-2, softmax and gate arithmetic) and
 //      computes counts, offsets and the stable (expert, token) permutation;
-//   3. cluster barrier; every CTA copies its share of the 2T permuted rows of
-//      x (converted to fp16 for int8 weights), reading the positions from CTA 0;
-//   4. cluster barrier, so CTA 0's shared memory outlives those reads.
-constexpr int kSmallCTAs = 8;
+//   3. cluster barrier; every CTA reads the positions it needs out of CTA 0's
+//      shared memory, arrives on the cluster barrier and writes the permuted
+//      rows of x (converted to fp16 for int8 weights). When one pass of the
+//      warps covers the tokens (T <= 64) and a lane's share of the slice fits
+//      kXU vectors, the x values loaded in step 1 are still in registers and
+//      each CTA stores its slice of both of a token's rows; otherwise the 2T
+//      rows are read from x again, eight 16-byte loads in flight per thread;
+//   4. wait on that barrier, so CTA 0's shared memory outlives those reads.
+// The cluster has 16 CTAs (above the portable 8; small_route_dispatch checks
+// once per device that it fits) because the loads and stores of steps 1 and 3
+// are bound by what few SMs keep in flight: with 8 CTAs the kernel took 13 us
+// at T = 64, d = 6144 on a B200, 3 us of it in the stores of step 3.
+constexpr int kSmallCTAs = 16;  // a non-portable cluster size: checked per device before use
 constexpr int kSmallMaxT = 128;
-constexpr int kSmallThreads = 256;
+constexpr int kSmallThreads = 512;
+constexpr int64_t kSmallMaxD = 65536;  // 2 * kSmallMaxT rows of d elements index in 32 bits
+constexpr int kXU = 2;                 // 16-byte x vectors per lane and token loaded together
+constexpr int kStageIt = (2 * kWrRows + kSmallThreads - 1) / kSmallThreads;  // router-row float4 per thread
 
 template <typename TX, bool F16 = false>
-__global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThreads)
+__global__ void __launch_bounds__(kSmallThreads)
     moe_route_dispatch_small_kernel(const TX* __restrict__ x, const float* __restrict__ wr,
                                     const float* __restrict__ bias, int64_t T, int64_t d, int32_t renormalize,
                                     int32_t* __restrict__ idx, float* __restrict__ gates,
@@ -489,7 +536,7 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
                                     TX* __restrict__ xp, uint32_t* __restrict__ status) {
   using namespace moe::sm100;
   constexpr int V = Vec<TX>::N;
-  __shared__ float part[kSmallMaxT][kE];  // this CTA's partial logits
+  __shared__ __align__(16) float part[kSmallMaxT][kE];  // this CTA's partial logits
   __shared__ int sel[kSmallMaxT][2];      // CTA 0: chosen experts
   __shared__ float sgate[kSmallMaxT][2];  // CTA 0: their gates
   __shared__ int pos[kSmallMaxT][2];      // CTA 0: permuted row of each (token, slot)
@@ -501,8 +548,15 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
   if (threadIdx.x < kE) cnt[threadIdx.x] = 0;
 
   // 1. Partial logits over this CTA's slice, kTokPerWarp tokens per warp pass.
+  //    Each lane issues its kXU x vectors of every token before the router
+  //    rows are staged, so the two loads overlap.
   const int64_t len = d / kSmallCTAs;
   const int64_t c_begin = static_cast<int64_t>(rank) * len;
+  // One pass over the tokens and one block of x vectors: the x values stay in
+  // registers for the copy in step 3 (decode shapes: T <= 64, d <= 6144 bf16).
+  const bool keep = T <= kWarps * kTokPerWarp && len <= kWrRows && len <= static_cast<int64_t>(kXU) * 32 * V;
+  uint4 raw[kXU][kTokPerWarp];
+  int64_t staged = -1;  // the slice chunk whose router rows wsm holds (the same in every thread)
   for (int64_t tb = static_cast<int64_t>(warp) * kTokPerWarp; tb < kSmallMaxT; tb += kWarps * kTokPerWarp) {
     // every warp runs the same number of passes (the __syncthreads below)
     const TX* rows[kTokPerWarp];
@@ -515,71 +569,104 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
       for (int e = 0; e < kE; ++e) acc[j][e] = 0.0f;
     for (int64_t cc = c_begin; cc < c_begin + len; cc += kWrRows) {
       const int rows_here = static_cast<int>(min(static_cast<int64_t>(kWrRows), c_begin + len - cc));
-      __syncthreads();
-      for (int q = threadIdx.x; q < rows_here * 2; q += blockDim.x) {
-        const int r = q >> 1;
-        wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] =
-            *reinterpret_cast<const float4*>(wr + (cc + r) * kE + (q & 1) * 4);
-      }
-      __syncthreads();
-      if (tb < T) {
-        for (int r0 = lane * V; r0 < rows_here; r0 += 32 * V) {
-          float xv[kTokPerWarp][V];
+      for (int xb = 0; xb < rows_here; xb += kXU * 32 * V) {
+        if (tb < T) {
 #pragma unroll
-          for (int j = 0; j < kTokPerWarp; ++j) Vec<TX>::load(rows[j] + cc + r0, xv[j]);
+          for (int u = 0; u < kXU; ++u) {
+            const int r0 = xb + (u * 32 + lane) * V;
+            if (r0 < rows_here)
 #pragma unroll
-          for (int i = 0; i < V; ++i) {
-            const int r = r0 + i;
-            const float4 a = wsm[(r * kE + (r / V) * 4) / 4];
-            const float4 b = wsm[(r * kE + (r / V) * 4) / 4 + 1];
-            const float w[kE] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+              for (int j = 0; j < kTokPerWarp; ++j) raw[u][j] = *reinterpret_cast<const uint4*>(rows[j] + cc + r0);
+          }
+        }
+        if (cc != staged) {  // a slice within kWrRows rows is staged once for all passes
+          float4 wv[kStageIt];  // every load issued before the first store
 #pragma unroll
-            for (int j = 0; j < kTokPerWarp; ++j)
+          for (int k = 0; k < kStageIt; ++k) {
+            const int q = threadIdx.x + k * kSmallThreads;
+            if (q < rows_here * 2) wv[k] = *reinterpret_cast<const float4*>(wr + (cc + (q >> 1)) * kE + (q & 1) * 4);
+          }
+          __syncthreads();
 #pragma unroll
-              for (int e = 0; e < kE; ++e) acc[j][e] = fmaf(xv[j][i], w[e], acc[j][e]);
+          for (int k = 0; k < kStageIt; ++k) {
+            const int q = threadIdx.x + k * kSmallThreads;
+            const int r = q >> 1;
+            if (q < rows_here * 2) wsm[(r * kE + (r / V) * 4 + (q & 1) * 4) / 4] = wv[k];
+          }
+          __syncthreads();
+          staged = cc;
+        }
+        if (tb < T) {
+#pragma unroll
+          for (int u = 0; u < kXU; ++u) {
+            const int r0 = xb + (u * 32 + lane) * V;
+            if (r0 < rows_here) {
+              float xv[kTokPerWarp][V];
+#pragma unroll
+              for (int j = 0; j < kTokPerWarp; ++j) Vec<TX>::unpack(raw[u][j], xv[j]);
+#pragma unroll
+              for (int i = 0; i < V; ++i) {
+                const int r = r0 + i;
+                const float4 a = wsm[(r * kE + (r / V) * 4) / 4];
+                const float4 b = wsm[(r * kE + (r / V) * 4) / 4 + 1];
+                const float w[kE] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+                  for (int e = 0; e < kE; ++e) acc[j][e] = fmaf(xv[j][i], w[e], acc[j][e]);
+              }
+            }
           }
         }
       }
     }
     if (tb < T) {
-#pragma unroll
-      for (int j = 0; j < kTokPerWarp; ++j)
-#pragma unroll
-        for (int e = 0; e < kE; ++e) acc[j][e] = warp_sum(acc[j][e]);
-      if (lane < kTokPerWarp) {
-#pragma unroll
-        for (int j = 0; j < kTokPerWarp; ++j)
-          if (lane == j)
-#pragma unroll
-            for (int e = 0; e < kE; ++e) part[tb + j][e] = acc[j][e];
-      }
+      // lane L: the warp's sum for token tb + L / 8, expert L % 8
+      static_assert(kTokPerWarp * kE == 32, "one (token, expert) value per lane");
+      part[tb + lane / kE][lane % kE] = warp_reduce_scatter(acc, lane);
     }
   }
   cluster_sync();
 
-  // 2. CTA 0: routing and the permutation.
+  // 2. CTA 0: routing and the permutation. Four threads per token each sum
+  //    a quarter of the CTAs' partials (in CTA order); the quarters are added
+  //    as (q0 + q1) + (q2 + q3), the same in all four lanes.
   if (rank == 0) {
-    const int t = threadIdx.x;
+    static_assert(kSmallThreads == 4 * kSmallMaxT && kSmallCTAs % 4 == 0, "four threads per token");
+    constexpr int kPer = kSmallCTAs / 4;
+    const int t = threadIdx.x >> 2, q = threadIdx.x & 3;
+    float sum[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) sum[e] = 0.0f;
     if (t < T) {
-      float l[kE], sum[kE];
+      float4 pa[kPer], pb[kPer];
 #pragma unroll
-      for (int e = 0; e < kE; ++e) {
-        l[e] = bias ? bias[e] : 0.0f;
-        sum[e] = 0.0f;
-      }
-      for (uint32_t c = 0; c < kSmallCTAs; ++c) {
-        const uint32_t at = mapa_shared(&part[t][0], c);
-#pragma unroll
-        for (int e = 0; e < kE; ++e) sum[e] += ld_shared_cluster_f32(at + 4 * e);
+      for (int c = 0; c < kPer; ++c) {
+        const uint32_t at = mapa_shared(&part[t][0], static_cast<uint32_t>(q * kPer + c));
+        pa[c] = ld_shared_cluster_f32x4(at);
+        pb[c] = ld_shared_cluster_f32x4(at + 16);
       }
 #pragma unroll
-      for (int e = 0; e < kE; ++e) l[e] += sum[e];
-      finalize_token(l, t, renormalize, idx, gates, cnt);
-      // finalize_token wrote idx / gates to global memory; keep this thread's copy
-      sel[t][0] = idx[2 * t];
-      sel[t][1] = idx[2 * t + 1];
-      sgate[t][0] = gates[2 * t];
-      sgate[t][1] = gates[2 * t + 1];
+      for (int c = 0; c < kPer; ++c) {
+        sum[0] += pa[c].x; sum[1] += pa[c].y; sum[2] += pa[c].z; sum[3] += pa[c].w;
+        sum[4] += pb[c].x; sum[5] += pb[c].y; sum[6] += pb[c].z; sum[7] += pb[c].w;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kE; ++e) sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], 1);
+#pragma unroll
+    for (int e = 0; e < kE; ++e) sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], 2);
+    if (t < T && q == 0) {
+      float l[kE];
+#pragma unroll
+      for (int e = 0; e < kE; ++e) l[e] = (bias ? bias[e] : 0.0f) + sum[e];
+      const Top2 r = route_token(l, renormalize);
+      sel[t][0] = r.e0;
+      sel[t][1] = r.e1;
+      sgate[t][0] = r.g0;
+      sgate[t][1] = r.g1;
+      atomicAdd(&cnt[r.e0], 1);
+      atomicAdd(&cnt[r.e1], 1);
     }
     __syncthreads();
     if (warp == 0) {
@@ -590,11 +677,6 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
         base[e] = off;
         off += cnt[e];
       }
-      if (lane < kE) {
-        counts[lane] = cnt[lane];
-        offsets[lane] = base[lane];
-      }
-      if (lane == 0) offsets[kE] = off;
       const unsigned lt = (1u << lane) - 1u;
       for (int t0 = 0; t0 < T; t0 += 32) {
         const int t = t0 + lane;
@@ -614,15 +696,6 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
           if (kDebugBounds && !(index_ok(pa, 2 * T) && index_ok(pb, 2 * T))) {
             atomicOr(status, kStatusBounds);
             pa = pb = -1;
-          } else {
-            perm_token[pa] = t;
-            perm_slot[pa] = 0;
-            perm_token[pb] = t;
-            perm_slot[pb] = 1;
-            slot_pos[2 * t] = pa;
-            slot_pos[2 * t + 1] = pb;
-            gate_perm[pa] = sgate[t][0];
-            gate_perm[pb] = sgate[t][1];
           }
           pos[t][0] = pa;
           pos[t][1] = pb;
@@ -631,29 +704,110 @@ __global__ void __cluster_dims__(kSmallCTAs, 1, 1) __launch_bounds__(kSmallThrea
     }
   }
   cluster_sync();
+  // CTA 0 stores the routing and the permutation to global memory now, off
+  // the path to the barrier above (nothing in this kernel reads them back).
+  if (rank == 0) {
+    const int i = threadIdx.x;
+    if (i < 2 * T) {
+      const int t = i >> 1, s = i & 1;
+      const int p = pos[t][s];
+      idx[i] = sel[t][s];
+      gates[i] = sgate[t][s];
+      if (p >= 0) {
+        slot_pos[i] = p;
+        perm_token[p] = t;
+        perm_slot[p] = s;
+        gate_perm[p] = sgate[t][s];
+      }
+    }
+    if (i < kE) {
+      int base = 0;
+      for (int e = 0; e < i; ++e) base += cnt[e];
+      counts[i] = cnt[i];
+      offsets[i] = base;
+    }
+    if (i == kE) offsets[kE] = static_cast<int32_t>(2 * T);
+  }
 
-  // 3. The permuted copy of x, rows spread over the cluster's warps.
-  const int64_t vec_per_row = d * static_cast<int64_t>(sizeof(TX)) / 16;
+  // 3. The permuted copy of x.
+  uint32_t f16_bad = 0;
+  if (keep) {
+    // From registers: each warp stores its tokens' slice of x into both of
+    // their permuted rows (positions read from CTA 0, lane l: token l/2, slot l%2).
+    const int64_t tb = static_cast<int64_t>(warp) * kTokPerWarp;
+    int p_lane = -1;
+    if (lane < 2 * kTokPerWarp && tb + lane / 2 < T)
+      p_lane = ld_shared_cluster_s32(mapa_shared(&pos[tb + lane / 2][lane & 1], 0));
+    cluster_arrive();  // this CTA is done with CTA 0's shared memory
+    uint4* dst = reinterpret_cast<uint4*>(xp);
+#pragma unroll
+    for (int j = 0; j < kTokPerWarp; ++j)
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int p = __shfl_sync(0xffffffffu, p_lane, 2 * j + s);
+        if (tb + j >= T || p < 0) continue;
+#pragma unroll
+        for (int u = 0; u < kXU; ++u) {
+          const int r0 = (u * 32 + lane) * V;
+          if (r0 >= len) continue;
+          const int64_t at = (static_cast<int64_t>(p) * d + c_begin + r0) / V;  // 16-byte vector index
+          if (F16) {
+            const uint4 h = bf16x8_to_f16x8(raw[u][j]);
+            f16_bad |= f16x8_nonfinite(h);
+            dst[at] = h;
+          } else {
+            dst[at] = raw[u][j];
+          }
+        }
+      }
+    if (F16 && f16_bad) atomicOr(status, kStatusFp16Range);
+    cluster_wait();  // CTA 0's shared memory stays until every CTA has read it
+    return;
+  }
+  // Otherwise: positions into this CTA's shared memory, then the 2T rows as
+  // 16-byte vectors read again from x, spread over all the cluster's threads.
+  if (rank != 0)
+    for (int i = threadIdx.x; i < 2 * T; i += blockDim.x)
+      (&pos[0][0])[i] = ld_shared_cluster_s32(mapa_shared(&pos[0][0] + i, 0));
+  cluster_arrive();  // this CTA is done with CTA 0's shared memory
+  __syncthreads();
+  // 32-bit indices: 2T * vec_per_row <= 2 * kSmallMaxT * kSmallMaxD / 4 < 2^31
+  const int vec_per_row = static_cast<int>(d * static_cast<int64_t>(sizeof(TX)) / 16);
   const uint4* src = reinterpret_cast<const uint4*>(x);
   uint4* dst = reinterpret_cast<uint4*>(xp);
-  uint32_t f16_bad = 0;
-  for (int64_t r = static_cast<int64_t>(rank) * kWarps + warp; r < 2 * T; r += kSmallCTAs * kWarps) {
-    const int64_t t = r >> 1;
-    const int p = ld_shared_cluster_s32(mapa_shared(&pos[t][r & 1], 0));
-    if (p < 0) continue;
-    for (int64_t c = lane; c < vec_per_row; c += 32) {
-      const uint4 v = src[t * vec_per_row + c];
+  const int total = 2 * static_cast<int>(T) * vec_per_row;
+  constexpr int stride = kSmallCTAs * kSmallThreads;
+  for (int i0 = static_cast<int>(rank) * kSmallThreads + threadIdx.x; i0 < total; i0 += 8 * stride) {
+    uint4 v[8];
+    int o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * stride;
+      o[u] = -1;
+      if (i < total) {
+        const int r = i / vec_per_row;
+        const int c = i - r * vec_per_row;
+        const int p = pos[r >> 1][r & 1];
+        if (p >= 0) {
+          v[u] = src[(r >> 1) * vec_per_row + c];
+          o[u] = p * vec_per_row + c;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (o[u] < 0) continue;
       if (F16) {
-        const uint4 h = bf16x8_to_f16x8(v);
+        const uint4 h = bf16x8_to_f16x8(v[u]);
         f16_bad |= f16x8_nonfinite(h);
-        dst[static_cast<int64_t>(p) * vec_per_row + c] = h;
+        dst[o[u]] = h;
       } else {
-        dst[static_cast<int64_t>(p) * vec_per_row + c] = v;
+        dst[o[u]] = v[u];
       }
     }
   }
   if (F16 && f16_bad) atomicOr(status, kStatusFp16Range);
-  cluster_sync();  // CTA 0's shared memory stays until every CTA has read it
+  cluster_wait();  // CTA 0's shared memory stays until every CTA has read it
 }
 
 template <typename TO>
@@ -857,27 +1011,80 @@ cudaError_t launch_dispatch(moe_dtype_t dtype, const void* x, int64_t T, int64_t
   return cudaGetLastError();
 }
 
-bool small_route_dispatch(int64_t T, const void* xp) { return T > 0 && T <= kSmallMaxT && xp != nullptr; }
+namespace {
+
+cudaLaunchConfig_t small_config(cudaLaunchAttribute* at, cudaStream_t s) {
+  at->id = cudaLaunchAttributeClusterDimension;
+  at->val.clusterDim.x = kSmallCTAs;
+  at->val.clusterDim.y = 1;
+  at->val.clusterDim.z = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(kSmallCTAs, 1, 1);
+  c.blockDim = dim3(kSmallThreads, 1, 1);
+  c.stream = s;
+  c.attrs = at;
+  c.numAttrs = 1;
+  return c;
+}
+
+// Allows the cluster size above the portable 8 and checks that one cluster
+// fits on this device; 0 when it does not (the two-kernel path is used then).
+template <typename TX, bool F16>
+int small_cluster_fits() {
+  auto kern = moe_route_dispatch_small_kernel<TX, F16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchAttribute at;
+  const cudaLaunchConfig_t c = small_config(&at, nullptr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &c) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n >= 1 ? 1 : 0;
+}
+
+template <typename TX, bool F16>
+cudaError_t launch_small(const TX* x, const float* w_router, const float* bias, int64_t T, int64_t d,
+                         int32_t renormalize, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
+                         int32_t* perm_token, int32_t* perm_slot, int32_t* slot_pos, float* gate_perm, TX* xp,
+                         uint32_t* status, cudaStream_t s) {
+  cudaLaunchAttribute at;
+  const cudaLaunchConfig_t c = small_config(&at, s);
+  return cudaLaunchKernelEx(&c, moe_route_dispatch_small_kernel<TX, F16>, x, w_router, bias, T, d, renormalize,
+                            idx, gates, counts, offsets, perm_token, perm_slot, slot_pos, gate_perm, xp, status);
+}
+
+}  // namespace
+
+bool small_route_dispatch(int64_t T, int64_t d, const void* xp) {
+  if (!(T > 0 && T <= kSmallMaxT && d <= kSmallMaxD && xp != nullptr)) return false;
+  const int ok = once_per_device(reinterpret_cast<const void*>(&small_route_dispatch), [](const void*) -> int {
+    return small_cluster_fits<float, false>() && small_cluster_fits<__nv_bfloat16, false>() &&
+                   small_cluster_fits<__nv_bfloat16, true>()
+               ? 1
+               : 0;
+  });
+  return ok == 1;
+}
 
 cudaError_t launch_route_dispatch_small(moe_dtype_t dtype, const void* x, const float* w_router, const float* bias,
                                         int64_t T, int64_t d, int32_t renormalize, int32_t* idx, float* gates,
                                         int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
                                         int32_t* slot_pos, float* gate_perm, void* xp, uint32_t* status,
                                         cudaStream_t s) {
-  const dim3 grid(kSmallCTAs), block(kSmallThreads);
   if (dtype == MOE_F32)
-    moe_route_dispatch_small_kernel<float><<<grid, block, 0, s>>>(
-        static_cast<const float*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets, perm_token,
-        perm_slot, slot_pos, gate_perm, static_cast<float*>(xp), status);
-  else if (dtype == MOE_BF16_INT8W)
-    moe_route_dispatch_small_kernel<__nv_bfloat16, true><<<grid, block, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets,
-        perm_token, perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), status);
-  else
-    moe_route_dispatch_small_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, bias, T, d, renormalize, idx, gates, counts, offsets,
-        perm_token, perm_slot, slot_pos, gate_perm, static_cast<__nv_bfloat16*>(xp), status);
-  return cudaGetLastError();
+    return launch_small<float, false>(static_cast<const float*>(x), w_router, bias, T, d, renormalize, idx, gates,
+                                      counts, offsets, perm_token, perm_slot, slot_pos, gate_perm,
+                                      static_cast<float*>(xp), status, s);
+  using B = __nv_bfloat16;
+  if (dtype == MOE_BF16_INT8W)
+    return launch_small<B, true>(static_cast<const B*>(x), w_router, bias, T, d, renormalize, idx, gates, counts,
+                                 offsets, perm_token, perm_slot, slot_pos, gate_perm, static_cast<B*>(xp), status, s);
+  return launch_small<B, false>(static_cast<const B*>(x), w_router, bias, T, d, renormalize, idx, gates, counts,
+                                offsets, perm_token, perm_slot, slot_pos, gate_perm, static_cast<B*>(xp), status, s);
 }
 
 cudaError_t launch_combine(moe_dtype_t dtype, const float* y, int64_t split_stride, int32_t splits,
