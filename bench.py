@@ -344,14 +344,17 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 def launches_per_step(wl, path):
     """Kernels of ours per step: router, dispatch (one cluster launch for both
     at T <= 128) and two GEMMs (the down projection's epilogue sums each
-    token's rows, so no combine kernel runs); with the automatic token-tile
-    choice on bf16 weights each GEMM launches both forms (the one not chosen
-    returns at once); above 1024 router blocks (T > 32768) a histogram scan
-    runs before the dispatch."""
+    token's rows, so no combine kernel runs). With the automatic token-tile
+    choice on bf16 weights a GEMM launches both 128-row forms (the one not
+    chosen returns at once), except the gate/up GEMM from 1024 tokens, which
+    runs 256-row tiles alone. Above 1024 router blocks (T > 32768) a histogram
+    scan runs before the dispatch."""
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
+    tall_gateup = both and wl.T >= 1024
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
     route = 1 if wl.T <= 128 else 2
-    return route + 2 + (2 if both else 0) + (1 if scan else 0)
+    gemms = (1 if tall_gateup else (2 if both else 1)) + (2 if both else 1)
+    return route + gemms + (1 if scan else 0)
 
 
 # ---------------------------------------------------------------- main --
@@ -427,7 +430,7 @@ def main():
     value = job_throughput(world, K, flops, t_max) / 1e12
     tok_s = job_throughput(world, K, T, t_max)
     wbytes = touched * 3 * d * f * (1 if wl.dtype == "bf16_int8w" else 2)
-    roofline = roofline_entry(wl, pk, stage_ms, touched, clocks)
+    roofline = roofline_entry(wl, pk, stage_ms, touched, clocks, a.path)
 
     e2e = None if a.no_e2e else run_e2e(a, moe, inp, run, out, flush, dist, dev, world, flops)
     int8 = skewed = None
@@ -538,7 +541,7 @@ def recorded_traffic(wl):
     return k["dram_read_bytes"] + k["dram_write_bytes"]
 
 
-def roofline_entry(wl, pk, stage_ms, touched, clocks):
+def roofline_entry(wl, pk, stage_ms, touched, clocks, path="auto"):
     """The gate/up GEMM is the dominant kernel (2/3 of the FLOPs; in the
     weight-stream form 2/3 of the weight bytes). A step here is milliseconds
     long and the timed region well under a second, so a tensor-bound fraction
@@ -562,8 +565,12 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks):
     dn = 4 * T * d * f / (dn_ms / 1e3) / 1e12
     wbytes = wl.E * 2 * d * f * esz
     act = 2 * T * d * 2 + 2 * T * f * 2
-    kern = ("gate/up expert GEMM, int8 weights, 256-row token tiles" if esz == 1 else
-            "gate/up expert GEMM, token tiles (single-CTA or CTA-pair form, chosen on the device)")
+    if esz == 1:
+        kern = "gate/up expert GEMM, int8 weights, 256-row token tiles"
+    elif T >= 1024 and path == "auto" and wl.dtype == "bf16":
+        kern = "gate/up expert GEMM, bf16, 256-row token tiles on single CTAs"
+    else:
+        kern = "gate/up expert GEMM, token tiles (single-CTA or CTA-pair form, chosen on the device)"
     out = {"bound": "tensor", "kernel": kern,
            "achieved": round(gu, 1), "peak": peak_t, "unit": "TFLOP/s", "frac": round(gu / peak_t, 4),
            "frac_sustained": round(gu / peak_s, 4), "peak_sustained": peak_s,

@@ -104,12 +104,14 @@ static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cf
                   Cfg<true, false, true>::SMEM <= 232448 && Cfg<false, false, true>::SMEM <= 232448,
               "shared memory above the per-block limit");
 
-template <int KIND, bool WS, bool W8, bool SHORT = false>
+// TALL: 256-row token tiles (always with int8 weights; bf16 gate/up for
+// larger batches, see launch_tc_gateup).
+template <int KIND, bool WS, bool W8, bool SHORT = false, bool TALL = W8 && !WS>
 __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     moe_expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                            const __grid_constant__ CUtensorMap tm_w1, const Params p) {
   static_assert(!SHORT || WS, "short tiles are a weight-stream form");
-  constexpr bool TALL = W8 && !WS;
+  static_assert(!TALL || !WS, "tall tiles are a token-tile form");
   constexpr int TROWS = TALL ? 2 * BM : (SHORT ? BM / 2 : BM);  // token rows per tile
   constexpr int NACC = TALL ? 1 : 2;         // accumulator buffers in flight
   using C = Cfg<W8, TALL, SHORT>;
@@ -533,11 +535,10 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
   }
 }
 
-template <int KIND, bool WS, bool W8, bool SHORT = false>
+template <int KIND, bool WS, bool W8, bool SHORT = false, bool TALL = W8 && !WS>
 cudaError_t launch_one(const TcGemmArgs& a, cudaStream_t stream) {
-  constexpr bool TALL = W8 && !WS;
   using C = Cfg<W8, TALL, SHORT>;
-  auto kern = moe_expert_gemm_kernel<KIND, WS, W8, SHORT>;
+  auto kern = moe_expert_gemm_kernel<KIND, WS, W8, SHORT, TALL>;
   const cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
 
@@ -613,7 +614,13 @@ cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s) {
                           : tc::launch_one<tc::GATEUP, true, false, true>(a, s);
   if (a.weight_stream)
     return a.int8_weights ? tc::launch_one<tc::GATEUP, true, true>(a, s) : tc::launch_one<tc::GATEUP, true, false>(a, s);
-  return a.int8_weights ? tc::launch_one<tc::GATEUP, false, true>(a, s) : tc::launch_one<tc::GATEUP, false, false>(a, s);
+  if (a.int8_weights) return tc::launch_one<tc::GATEUP, false, true>(a, s);
+  // bf16 gate/up in 256-row tiles: each weight tile feeds two M = 128 MMAs on
+  // one SM, which halves the weight bytes each SM reads from L2 per FLOP
+  // (measured gate/up T = 1024 / 4096 / 8192: 1.71 / 5.64-5.68 / 11.0-11.5 ms
+  // against 1.78 / 5.84-5.95 / 11.4-12.0 ms for the CTA-pair form).
+  return a.tall_tiles ? tc::launch_one<tc::GATEUP, false, false, false, true>(a, s)
+                      : tc::launch_one<tc::GATEUP, false, false>(a, s);
 }
 
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s) {

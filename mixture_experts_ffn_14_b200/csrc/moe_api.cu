@@ -408,7 +408,21 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
       }
       return cudaSuccess;
     };
-    MOE_TRY(launch_gemm(g, false));
+    // bf16 gate/up under AUTO with at least kTallMinT tokens (256 rows per
+    // expert on average): 256-row tiles on single CTAs, which beat both
+    // 128-row forms there (measured gate/up, two runs: T = 768 1.38 against
+    // 1.33-1.34 ms, so not below; T = 1024 1.77-1.95 against 1.87-1.97;
+    // T = 4096 5.19-5.59 against 5.67-5.80). The down projection keeps the
+    // choice above: its epilogue, which 256-row tiles cannot overlap with the
+    // next tile, is heavier.
+    if (auto_tt && !gather_x && T >= kTallMinT) {
+      TcGemmArgs gt = g;
+      gt.tall_tiles = true;
+      gt.select = 0;
+      MOE_TRY(launch_tc_gateup(gt, stream));
+    } else {
+      MOE_TRY(launch_gemm(g, false));
+    }
     MOE_TRY(mark(3));
     TcGemmArgs g2 = g;
     g2.x = h;

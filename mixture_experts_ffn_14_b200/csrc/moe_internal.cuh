@@ -17,6 +17,7 @@ namespace moe {
 constexpr int kE = 8;              // experts (this version)
 constexpr int kK = 2;              // experts per token
 constexpr int kRouteTokens = 32;   // tokens per router / dispatch CTA
+constexpr int64_t kTallMinT = 1024;  // bf16 gate/up under MOE_PATH_AUTO: 256-row tiles from this many tokens
 
 // Device status word bits (set with atomicOr; 0 = no failure recorded).
 enum : uint32_t {
@@ -132,6 +133,7 @@ struct TcGemmArgs {
   uint32_t* status;
   int32_t n_experts;        // experts in the weight arrays (0 = kE); experts past it have no rows
   bool short_tiles;         // weight-stream: tiles of at most 64 tokens, deeper weight ring
+  bool tall_tiles;          // bf16 GATEUP token tiles: 256-row tiles on single CTAs (int8 always uses them)
   // DOWN token tiles: the combine in the epilogue (out[t] = sum of the two
   // gate-scaled rows of token t, in fixed order). combine_count == nullptr:
   // the epilogue only writes Y and a separate combine kernel runs.

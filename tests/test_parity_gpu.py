@@ -246,6 +246,21 @@ def test_int8_every_code_converts_exactly(path):
 
 # ------------------------------------------------------- determinism etc --
 
+@pytest.mark.parametrize("T", [1024, 1100, 2100])
+def test_tall_bf16_gateup_tiles(T):
+    # From 1024 tokens the automatic path runs the bf16 gate/up GEMM in 256-row
+    # tiles (two M = 128 MMAs per weight tile). Experts of 1-255 rows beyond
+    # a multiple of 256 end in a partial tile: one MMA per step when it has at
+    # most 128 rows. Each element of H accumulates the same 16-deep K steps in
+    # the same order as in 128-row tiles, so H must equal the single-CTA
+    # 128-row form bit for bit; H and out must match the oracle.
+    inp = small_bf16(T, d=512, f=1024, seed=T)
+    a = run_gpu(inp, path=moe.MOE_PATH_AUTO)
+    b = run_gpu(inp, path=moe.MOE_PATH_TOKEN_TILE_SINGLE)
+    assert torch.equal(a["h"], b["h"])
+    full_check(inp, a, tokens=np.arange(0, T, 7))
+
+
 def test_bitwise_determinism_and_streams():
     inp = small_bf16(333, seed=31)
     a = run_gpu(inp)
