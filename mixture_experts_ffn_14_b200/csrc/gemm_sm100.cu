@@ -72,7 +72,12 @@ struct Cfg {
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
-  static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : 256;
+  // bf16 256-row tiles: a second set of four epilogue warps (warps 8-11) takes
+  // rows 128-255 while warps 4-7 take rows 0-127, halving the epilogue that
+  // these tiles cannot overlap with the next tile's main loop (gate/up, median
+  // of four alternating runs: T = 4096 5.685 -> 5.600 ms, T = 1024 1.711 -> 1.703).
+  static constexpr int EPI_WARPS = (TALL && !W8) ? 8 : 4;
+  static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : (TALL ? 384 : 256);
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
@@ -107,7 +112,7 @@ static_assert(Cfg<true, true>::SMEM <= 232448 && Cfg<true>::SMEM <= 232448 && Cf
 // TALL: 256-row token tiles (always with int8 weights; bf16 gate/up for
 // larger batches, see launch_tc_gateup).
 template <int KIND, bool WS, bool W8, bool SHORT = false, bool TALL = W8 && !WS>
-__global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
+__global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
     moe_expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                            const __grid_constant__ CUtensorMap tm_w1, const Params p) {
   static_assert(!SHORT || WS, "short tiles are a weight-stream form");
@@ -152,11 +157,12 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 128);
+      mbar_init(&tempty_bar[b], 32 * C::EPI_WARPS);
     }
     for (int i = 0; i < kTileQS; ++i) {
       mbar_init(&qfull_bar[i], 1);
-      mbar_init(&qempty_bar[i], 1 + 4 + (W8 ? C::CONVERT_WARPS : 0));  // MMA, epilogue warps, converter warps
+      // MMA thread, epilogue warps, converter warps
+      mbar_init(&qempty_bar[i], 1 + C::EPI_WARPS + (W8 ? C::CONVERT_WARPS : 0));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -392,9 +398,11 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       }
     mma_done:;
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 4 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue --
-    const int q = warp - 4;  // TMEM lanes 32q .. 32q+31
+    const int q = warp % 4;  // TMEM lanes 32q .. 32q+31
+    const bool split = C::EPI_WARPS == 8;  // warps 8-11 take rows 128-255 of a tall tile
+    const bool upper = split && warp >= 8;
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
@@ -414,8 +422,8 @@ __global__ void __launch_bounds__(Cfg<W8>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * 256;
       if (!WS) {
-        epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, min(t.rows, BM));
-        if (TALL && t.rows > BM)  // rows 128..255 of a tall tile: accumulator columns 256..511
+        if (!upper) epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, min(t.rows, BM));
+        if (TALL && t.rows > BM && (upper || !split))  // rows 128..255: accumulator columns 256..511
           epilogue_token_rows<KIND, W8>(p, t, tbase + 256, 32 * q + lane, t.row0 + BM, t.rows - BM);
       } else {
         // Weight-stream: TMEM lane = output column, TMEM column = token.
