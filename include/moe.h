@@ -99,10 +99,15 @@ typedef enum {
 
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
  * down projection) when the average tokens per expert is small (T <= 256),
- * else token tiles (tokens on the MMA M side), where the device chooses from
- * the expert counts between 128-token tiles on single CTAs and 256-token tiles
- * on CTA pairs (cta_group::2). TOKEN_TILE forces the pair form,
- * TOKEN_TILE_SINGLE the single-CTA form. All compute the same result. */
+ * else token tiles (tokens on the MMA M side). With bf16 weights the gate/up
+ * GEMM then runs 256-token tiles on single CTAs from T = 1024 on; below that,
+ * and for the down GEMM, the device chooses from the expert counts between
+ * 128-token tiles on single CTAs and 256-token tiles on CTA pairs
+ * (cta_group::2). int8 weights take 256-token tiles on single CTAs.
+ * TOKEN_TILE forces the pair form, TOKEN_TILE_SINGLE the single-CTA form
+ * (128-token tiles for bf16). All compute the same result within rounding;
+ * each H element accumulates the same K steps in the same order in every
+ * token-tile form. */
 typedef enum {
   MOE_PATH_AUTO = 0,
   MOE_PATH_TOKEN_TILE = 1,
