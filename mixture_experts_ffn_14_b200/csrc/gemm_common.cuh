@@ -449,30 +449,34 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
   const bool valid = r < nvalid;
   const int64_t row = row_base + r;
   if (KIND == GATEUP) {
+    // Columns per step: 16 with int8 weights, whose kernel runs 640 threads
+    // (at most 96 registers each), 32 otherwise.
+    constexpr int CW = W8 ? 16 : 32;
     uint16_t* hout = static_cast<uint16_t*>(p.out);
     uint32_t f16_bad = 0;  // int8 weights: an H value beyond the fp16 range
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 32) {
-      // int8 weights: the chunk's 32 gate and 32 up channel scales as eight
-      // 16-byte loads (the same addresses in every lane), issued before the
-      // TMEM load so that their latency overlaps it.
-      uint32_t sg[16], su[16];
+    for (int c = 0; c < 128; c += CW) {
+      // int8 weights: the chunk's gate and up channel scales as 16-byte loads
+      // (the same addresses in every lane), issued before the TMEM load so
+      // that their latency overlaps it.
+      uint32_t sg[CW / 2], su[CW / 2];
       if (W8) {
         const int64_t sc = static_cast<int64_t>(t.e) * p.N + t.n0 + c;
         const uint4* a = reinterpret_cast<const uint4*>(p.s0 + sc);
         const uint4* b = reinterpret_cast<const uint4*>(p.s1 + sc);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < CW / 8; ++v) {
           const uint4 x = __ldg(a + v), y = __ldg(b + v);
           sg[4 * v] = x.x; sg[4 * v + 1] = x.y; sg[4 * v + 2] = x.z; sg[4 * v + 3] = x.w;
           su[4 * v] = y.x; su[4 * v + 1] = y.y; su[4 * v + 2] = y.z; su[4 * v + 3] = y.w;
         }
       }
-      uint32_t g[32], u[32];
-      tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
-      uint32_t packed[16];
+      uint32_t g[CW], u[CW];
+      if constexpr (CW == 16) tmem_ld16x2(tbase + c, tbase + 128 + c, g, u);
+      else tmem_ld32x2(tbase + c, tbase + 128 + c, g, u);
+      uint32_t packed[CW / 2];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
+      for (int j = 0; j < CW; j += 2) {
         float g0 = __uint_as_float(g[j]), g1 = __uint_as_float(g[j + 1]);
         float u0 = __uint_as_float(u[j]), u1 = __uint_as_float(u[j + 1]);
         if (W8) {  // bf16 pair (lo = column j, hi = j + 1) -> fp32 by a shift
@@ -489,7 +493,7 @@ __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile&
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(hout + row * p.N + t.n0 + c);
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
+        for (int v = 0; v < CW / 8; ++v)
           dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       }
     }

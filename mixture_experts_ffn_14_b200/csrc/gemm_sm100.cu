@@ -72,12 +72,14 @@ struct Cfg {
   static constexpr int RING_BYTES = STAGES * SLOT_BYTES + CSTAGES * W_BYTES;
   static constexpr int CONVERT_THREADS = 256;
   static constexpr int CONVERT_WARPS = CONVERT_THREADS / 32;
-  // bf16 256-row tiles: a second set of four epilogue warps (warps 8-11) takes
-  // rows 128-255 while warps 4-7 take rows 0-127, halving the epilogue that
-  // these tiles cannot overlap with the next tile's main loop (gate/up, median
-  // of four alternating runs: T = 4096 5.685 -> 5.600 ms, T = 1024 1.711 -> 1.703).
-  static constexpr int EPI_WARPS = (TALL && !W8) ? 8 : 4;
-  static constexpr int THREADS = W8 ? 256 + CONVERT_THREADS : (TALL ? 384 : 256);
+  // 256-row tiles: a second set of four epilogue warps (warps 8-11) takes rows
+  // 128-255 while warps 4-7 take rows 0-127, halving the epilogue that these
+  // tiles cannot overlap with the next tile's main loop. bf16 gate/up, median
+  // of four alternating runs: T = 4096 5.685 -> 5.600 ms, T = 1024 1.711 ->
+  // 1.703. int8 (640 threads, converters in warps 12-19; median of three
+  // alternating runs): step T = 1024 2.959 -> 2.880 ms, T = 4096 9.587 -> 9.265.
+  static constexpr int EPI_WARPS = TALL ? 8 : 4;
+  static constexpr int THREADS = 128 + 32 * EPI_WARPS + (W8 ? CONVERT_THREADS : 0);
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
 };
@@ -486,7 +488,7 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
         acc_phase ^= 1;
       }
     }
-  } else if (W8 && warp >= 8) {
+  } else if (W8 && warp >= 4 + C::EPI_WARPS) {
     // ----------------------------------------------- int8 -> fp16 convert --
     // Staging: two int8 boxes [64 K][128 N] (row = 128 B) in TMA slot `stage`.
     // Target: converted slot `cstage`, four fp16 chunks [64 K][64 N] with the
@@ -494,8 +496,8 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
     constexpr int GROUPS = conv_groups(WS);
     constexpr int GWARPS = C::CONVERT_WARPS / GROUPS;  // warps per group
     constexpr int GTHREADS = 32 * GWARPS;
-    const int grp = (warp - 8) / GWARPS;
-    const int ct = threadIdx.x - 256 - grp * GTHREADS;  // 0 .. GTHREADS-1 within the group
+    const int grp = (warp - 4 - C::EPI_WARPS) / GWARPS;
+    const int ct = threadIdx.x - 128 - 32 * C::EPI_WARPS - grp * GTHREADS;  // 0 .. GTHREADS-1 within the group
     int n = 0;  // K-block step of this CTA, counted over all its tiles
     Tile t;
     for (int i = 0;; ++i) {
