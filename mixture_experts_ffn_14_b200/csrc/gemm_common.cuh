@@ -443,19 +443,20 @@ __device__ __forceinline__ void ws_combine_arrive(const Params& p, const Tile& t
 // columns. GATEUP: columns 0..127 gate, 128..255 up -> H[row, n0 + c] (bf16; fp16 with int8 weights).
 // DOWN: 256 output columns -> fp32 Y[split, row, n0 + c] = acc * gate[row],
 // then (combine_count set) the combine above.
-template <int KIND, bool W8>
+// GATEUP: H columns [c_begin, c_end) of the tile (a warp may take part of
+// them); CW columns per TMEM load: 16 where the kernel runs 640 threads (at
+// most 96 registers each), 32 otherwise.
+template <int KIND, bool W8, int CW = (W8 ? 16 : 32)>
 __device__ __forceinline__ void epilogue_token_rows(const Params& p, const Tile& t, uint32_t tbase, int r,
-                                                    int64_t row_base, int nvalid) {
+                                                    int64_t row_base, int nvalid, int c_begin = 0, int c_end = 128) {
   const bool valid = r < nvalid;
   const int64_t row = row_base + r;
   if (KIND == GATEUP) {
-    // Columns per step: 16 with int8 weights, whose kernel runs 640 threads
-    // (at most 96 registers each), 32 otherwise.
-    constexpr int CW = W8 ? 16 : 32;
+    static_assert(CW == 16 || CW == 32, "16 or 32 columns per TMEM load");
     uint16_t* hout = static_cast<uint16_t*>(p.out);
     uint32_t f16_bad = 0;  // int8 weights: an H value beyond the fp16 range
 #pragma unroll 1
-    for (int c = 0; c < 128; c += CW) {
+    for (int c = c_begin; c < c_end; c += CW) {
       // int8 weights: the chunk's gate and up channel scales as 16-byte loads
       // (the same addresses in every lane), issued before the TMEM load so
       // that their latency overlaps it.

@@ -78,7 +78,10 @@ struct Cfg {
   // of four alternating runs: T = 4096 5.685 -> 5.600 ms, T = 1024 1.711 ->
   // 1.703. int8 (640 threads, converters in warps 12-19; median of three
   // alternating runs): step T = 1024 2.959 -> 2.880 ms, T = 4096 9.587 -> 9.265.
-  static constexpr int EPI_WARPS = TALL ? 8 : 4;
+  // bf16 256-row tiles run 16 epilogue warps (640 threads): each set of four
+  // takes one 128-row half and one 64-column half of H (gate/up, median of
+  // three alternating runs: T = 4096 5.468 -> 5.350 ms, T = 8192 10.53 -> 10.31).
+  static constexpr int EPI_WARPS = TALL ? (W8 ? 8 : 16) : 4;
   static constexpr int THREADS = 128 + 32 * EPI_WARPS + (W8 ? CONVERT_THREADS : 0);
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
@@ -403,8 +406,15 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
   } else if (warp >= 4 && warp < 4 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue --
     const int q = warp % 4;  // TMEM lanes 32q .. 32q+31
-    const bool split = C::EPI_WARPS == 8;  // warps 8-11 take rows 128-255 of a tall tile
-    const bool upper = split && warp >= 8;
+    // Tall tiles: warps 4-7 and 8-11 take rows 0-127 and 128-255; with 16
+    // epilogue warps (bf16), warps 12-19 do the same for the second half of
+    // the H columns, the first eight for the first half.
+    const bool split = C::EPI_WARPS >= 8;
+    const int set = (warp - 4) / 4;
+    const bool upper = split && (set & 1) != 0;
+    const int c_half = C::EPI_WARPS == 16 ? (set >> 1) : -1;
+    const int c_begin = c_half < 0 ? 0 : 64 * c_half, c_end = c_half < 0 ? 128 : c_begin + 64;
+    constexpr int ECW = (W8 || C::EPI_WARPS == 16) ? 16 : 32;
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile t;
@@ -424,9 +434,11 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * 256;
       if (!WS) {
-        if (!upper) epilogue_token_rows<KIND, W8>(p, t, tbase, 32 * q + lane, t.row0, min(t.rows, BM));
+        if (!upper)
+          epilogue_token_rows<KIND, W8, ECW>(p, t, tbase, 32 * q + lane, t.row0, min(t.rows, BM), c_begin, c_end);
         if (TALL && t.rows > BM && (upper || !split))  // rows 128..255: accumulator columns 256..511
-          epilogue_token_rows<KIND, W8>(p, t, tbase + 256, 32 * q + lane, t.row0 + BM, t.rows - BM);
+          epilogue_token_rows<KIND, W8, ECW>(p, t, tbase + 256, 32 * q + lane, t.row0 + BM, t.rows - BM, c_begin,
+                                             c_end);
       } else {
         // Weight-stream: TMEM lane = output column, TMEM column = token.
         const int ntok = ((t.rows + 15) / 16) * 16;
