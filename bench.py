@@ -346,11 +346,11 @@ def launches_per_step(wl, path):
     at T <= 128) and two GEMMs (the down projection's epilogue sums each
     token's rows, so no combine kernel runs). With the automatic token-tile
     choice on bf16 weights a GEMM launches both 128-row forms (the one not
-    chosen returns at once), except the gate/up GEMM from 1024 tokens, which
+    chosen returns at once), except the gate/up GEMM from 512 tokens, which
     runs 256-row tiles alone. Above 1024 router blocks (T > 32768) a histogram
     scan runs before the dispatch."""
     both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
-    tall_gateup = both and wl.T >= 1024
+    tall_gateup = both and wl.T >= 512
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
     route = 1 if wl.T <= 128 else 2
     gemms = (1 if tall_gateup else (2 if both else 1)) + (2 if both else 1)
@@ -567,7 +567,7 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks, path="auto"):
     act = 2 * T * d * 2 + 2 * T * f * 2
     if esz == 1:
         kern = "gate/up expert GEMM, int8 weights, 256-row token tiles"
-    elif T >= 1024 and path == "auto" and wl.dtype == "bf16":
+    elif T >= 512 and path == "auto" and wl.dtype == "bf16":
         kern = "gate/up expert GEMM, bf16, 256-row token tiles on single CTAs"
     else:
         kern = "gate/up expert GEMM, token tiles (single-CTA or CTA-pair form, chosen on the device)"

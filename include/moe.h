@@ -100,7 +100,7 @@ typedef enum {
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
  * down projection) when the average tokens per expert is small (T <= 256),
  * else token tiles (tokens on the MMA M side). With bf16 weights the gate/up
- * GEMM then runs 256-token tiles on single CTAs from T = 1024 on; below that,
+ * GEMM then runs 256-token tiles on single CTAs from T = 512 on; below that,
  * and for the down GEMM, the device chooses from the expert counts between
  * 128-token tiles on single CTAs and 256-token tiles on CTA pairs
  * (cta_group::2). int8 weights take 256-token tiles on single CTAs.

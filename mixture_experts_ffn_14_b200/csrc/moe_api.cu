@@ -408,13 +408,13 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
       }
       return cudaSuccess;
     };
-    // bf16 gate/up under AUTO with at least kTallMinT tokens (256 rows per
+    // bf16 gate/up under AUTO with at least kTallMinT tokens (128 rows per
     // expert on average): 256-row tiles on single CTAs, which beat both
-    // 128-row forms there (measured gate/up, two runs: T = 768 1.38 against
-    // 1.33-1.34 ms, so not below; T = 1024 1.77-1.95 against 1.87-1.97;
-    // T = 4096 5.19-5.59 against 5.67-5.80). The down projection keeps the
-    // choice above: its epilogue, which 256-row tiles cannot overlap with the
-    // next tile, is heavier.
+    // 128-row forms there (measured gate/up with sixteen epilogue warps, two
+    // runs: T = 384 1.11 against 1.03 ms, so not below; T = 512 1.20 against
+    // 1.21; T = 768 1.31 against 1.34-1.36; T = 4096 5.15-5.39 against
+    // 5.67-5.80 before). The down projection keeps the choice above: its
+    // epilogue, which 256-row tiles cannot overlap with the next tile, is heavier.
     if (auto_tt && !gather_x && T >= kTallMinT) {
       TcGemmArgs gt = g;
       gt.tall_tiles = true;

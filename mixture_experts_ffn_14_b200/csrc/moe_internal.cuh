@@ -17,7 +17,7 @@ namespace moe {
 constexpr int kE = 8;              // experts (this version)
 constexpr int kK = 2;              // experts per token
 constexpr int kRouteTokens = 32;   // tokens per router / dispatch CTA
-constexpr int64_t kTallMinT = 1024;  // bf16 gate/up under MOE_PATH_AUTO: 256-row tiles from this many tokens
+constexpr int64_t kTallMinT = 512;  // bf16 gate/up under MOE_PATH_AUTO: 256-row tiles from this many tokens
 
 // Device status word bits (set with atomicOr; 0 = no failure recorded).
 enum : uint32_t {

@@ -50,13 +50,14 @@ def test_launch_count_rule():
     from mixture_experts_ffn_14_b200 import workloads as W
 
     # The down projection's epilogue sums each token's rows: no combine kernel.
-    # bf16 gate/up from 1024 tokens: 256-row tiles alone; down: both 128-row forms
+    # bf16 gate/up from 512 tokens: 256-row tiles alone; down: both 128-row forms
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "auto") == 5
     import dataclasses
     assert bench.launches_per_step(W.WORKLOADS["decode"], "auto") == 3   # router + dispatch in one launch
     assert bench.launches_per_step(W.WORKLOADS["int8"], "auto") == 4
     assert bench.launches_per_step(W.WORKLOADS["prefill"], "token_tile") == 4
     assert bench.launches_per_step(W.WORKLOADS["skewed"], "auto") == 5
-    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=512), "auto") == 6
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=384), "auto") == 6
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=512), "auto") == 5
     big = dataclasses.replace(W.WORKLOADS["prefill"], T=40000)   # > 1024 router blocks: + scan
     assert bench.launches_per_step(big, "auto") == 6
