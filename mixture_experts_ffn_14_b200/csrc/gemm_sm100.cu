@@ -255,7 +255,11 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
         int32_t rtok[4] = {0, 0, 0, 0};
         if (G) gather_rows(p, t, t.row0 + 4 * lane, rtok);
         const int nbox_x = WS ? (t.rows + XBOX_ROWS_WS - 1) / XBOX_ROWS_WS : 1;
-        const uint32_t xbytes = WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : C::XS_BYTES;
+        // A 256-row tile of at most 128 rows (the last of an expert) loads only
+        // the first activation box: its second MMA is skipped. Gate/up T = 512,
+        // two runs: 1.162 / 1.162 ms against 1.181 / 1.181 with both boxes.
+        const uint32_t xbytes =
+            WS ? nbox_x * XBOX_ROWS_WS * BK * 2 : ((TALL && !G && t.rows <= BM) ? X_BYTES : C::XS_BYTES);
         const uint32_t wbytes = W8 ? W8_BYTES : W_BYTES;
         for (int kb = 0; kb < p.kb_per_split; ++kb) {
           int ok = 1;
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(Cfg<W8, TALL, SHORT>::THREADS, 1)
                 tma_load_2d(xs + b * XBOX_ROWS_WS * 128, &tm_x, &full_bar[stage], k0, t.row0 + b * XBOX_ROWS_WS);
             } else if (!G) {
               tma_load_2d(xs, &tm_x, &full_bar[stage], k0, t.row0);
-              if (TALL) tma_load_2d(xs + X_BYTES, &tm_x, &full_bar[stage], k0, t.row0 + BM);
+              if (TALL && t.rows > BM) tma_load_2d(xs + X_BYTES, &tm_x, &full_bar[stage], k0, t.row0 + BM);
             }
             if (W8) {
               if (KIND == GATEUP) {
