@@ -341,6 +341,17 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
     return world * steps * work_per_step / (t_max_ms / 1e3)
 
 
+def weight_stream_form(wl, path):
+    """Whether the GEMMs run in the weight-stream orientation: forced, or on the
+    automatic path for small batches (T <= 256 with int8 weights, T <= 128 with
+    bf16 weights; the library's choice)."""
+    if path == "weight_stream":
+        return True
+    if path != "auto":
+        return False
+    return wl.T <= (256 if wl.dtype == "bf16_int8w" else 128)
+
+
 def launches_per_step(wl, path):
     """Kernels of ours per step: router, dispatch (one cluster launch for both
     at T <= 128) and two GEMMs (the down projection's epilogue sums each
@@ -349,7 +360,7 @@ def launches_per_step(wl, path):
     chosen returns at once), except the gate/up GEMM from 512 tokens, which
     runs 256-row tiles alone. Above 1024 router blocks (T > 32768) a histogram
     scan runs before the dispatch."""
-    both = path == "auto" and wl.dtype == "bf16" and wl.T > 256
+    both = path == "auto" and wl.dtype == "bf16" and not weight_stream_form(wl, path)
     tall_gateup = both and wl.T >= 512
     scan = (wl.T + 31) // 32 > 1024          # block-histogram scan before the dispatch
     route = 1 if wl.T <= 128 else 2
@@ -551,7 +562,7 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks, path="auto"):
     T, d, f = wl.T, wl.d, wl.f
     gu_ms, dn_ms = stage_ms["gate_up_gemm"], stage_ms["down_gemm"]
     esz = 1 if wl.dtype == "bf16_int8w" else 2
-    if T <= 256:   # weight-stream form: HBM bound
+    if weight_stream_form(wl, path):   # weight-stream form: HBM bound
         gu_bytes = touched * 2 * d * f * esz
         gu = gu_bytes / (gu_ms / 1e3) / 1e9
         dn = touched * d * f * esz / (dn_ms / 1e3) / 1e9

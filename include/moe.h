@@ -98,8 +98,9 @@ typedef enum {
 } moe_activation_t;
 
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
- * down projection) when the average tokens per expert is small (T <= 256),
- * else token tiles (tokens on the MMA M side). With bf16 weights the gate/up
+ * down projection) when the average tokens per expert is small (T <= 128 with
+ * bf16 weights, T <= 256 with int8 weights; measured crossovers), else token
+ * tiles (tokens on the MMA M side). With bf16 weights the gate/up
  * GEMM then runs 256-token tiles on single CTAs from T = 512 on; below that,
  * and for the down GEMM, the device chooses from the expert counts between
  * 128-token tiles on single CTAs and 256-token tiles on CTA pairs

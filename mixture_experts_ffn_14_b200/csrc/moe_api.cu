@@ -157,13 +157,18 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, 
   return r == CUDA_SUCCESS;
 }
 
-bool use_weight_stream(int64_t T, moe_path_t path) {
+bool use_weight_stream(int64_t T, moe_path_t path, moe_dtype_t dtype) {
   if (path == MOE_PATH_WEIGHT_STREAM) return true;
   if (path == MOE_PATH_TOKEN_TILE || path == MOE_PATH_TOKEN_TILE_SINGLE) return false;
-  // Average 2T/8 token slots per expert: at <= 64 (T <= 256) a 128-row token
-  // tile would be mostly padding, while weight-stream tiles take the tokens on
-  // the MMA N side and read each weight byte once.
-  return T <= 256;
+  // Weight-stream tiles take the tokens on the MMA N side and read each weight
+  // byte once; a 128-row token tile of a small batch is mostly padding. Where
+  // the crossover lies was measured (interleaved runs at the Grok-1 shape, step
+  // ms, weight-stream against 128-row token tiles): int8 weights keep the
+  // weight-stream form up to T = 256 (T = 256: 1.76 against 1.97); bf16 weights
+  // only up to T = 128 (T = 64: 1.62 against 1.65; T = 160: 1.80 against 1.74;
+  // T = 256: 2.11 against 1.67, where the weight-stream down projection's
+  // split-K costs most).
+  return T <= (dtype == MOE_BF16_INT8W ? 256 : 128);
 }
 
 // Split-K factor of the token-tile down projection. Its tiles are long (K = f)
@@ -219,7 +224,7 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   WorkspaceLayout L{};
   const int64_t rows = 2 * T;
   L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
-  L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path);
+  L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path, dtype);
   L.tile_path = dtype != MOE_F32 && !L.weight_stream;
   if (dtype == MOE_F32) {
     L.splits = 1;
@@ -634,10 +639,12 @@ bool experts_sizes_ok(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype_t dt
 ExpertsLayout plan_experts(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype_t dtype, moe_path_t path,
                            int32_t down_splits) {
   ExpertsLayout L{};
-  // Weight-stream tiles when the local experts hold few rows on average
-  // (<= 64, as in the whole-layer choice), token tiles otherwise.
+  // Weight-stream tiles when the local experts hold few rows on average (as in
+  // the whole-layer choice: <= 64 with int8 weights, <= 32 with bf16), token
+  // tiles otherwise.
+  const int64_t ws_rows = dtype == MOE_BF16_INT8W ? 64 : 32;
   L.weight_stream = dtype != MOE_F32 && (path == MOE_PATH_WEIGHT_STREAM ||
-                                         (path == MOE_PATH_AUTO && R <= 64 * static_cast<int64_t>(n)));
+                                         (path == MOE_PATH_AUTO && R <= ws_rows * static_cast<int64_t>(n)));
   const int64_t kblocks = f / 64;
   if (down_splits > 0) {
     L.splits = kblocks % down_splits == 0 && dtype != MOE_F32 ? down_splits : (down_splits == 1 ? 1 : -1);

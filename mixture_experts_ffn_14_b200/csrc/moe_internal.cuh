@@ -51,7 +51,7 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
                                int32_t down_splits, bool h_external);
 
 // Host: which kernel family a call uses.
-bool use_weight_stream(int64_t T, moe_path_t path);
+bool use_weight_stream(int64_t T, moe_path_t path, moe_dtype_t dtype);
 int32_t choose_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested);
 
 // ---- launchers (return cudaSuccess or the launch error) --------------------

@@ -60,6 +60,15 @@ def test_bf16_parity_all_paths(T, path):
     full_check(inp, run_gpu(inp, path=path))
 
 
+@pytest.mark.parametrize("T", [128, 129, 200, 256, 257])
+def test_bf16_automatic_form_boundary(T):
+    # The automatic path runs bf16 weights in the weight-stream form up to 128
+    # tokens and in token tiles above (both 128-row forms launched, one chosen
+    # on the device; 256-row gate/up tiles from 512).
+    inp = small_bf16(T, seed=70 + T)
+    full_check(inp, run_gpu(inp, path=moe.MOE_PATH_AUTO))
+
+
 # Row gather (moe_options_t.row_gather): token tiles read the gate/up operand
 # rows from x with TMA four-row gathers instead of the dispatch stage's copy.
 TT_PATHS = [moe.MOE_PATH_TOKEN_TILE, moe.MOE_PATH_TOKEN_TILE_SINGLE, moe.MOE_PATH_AUTO]

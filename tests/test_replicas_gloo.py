@@ -59,5 +59,10 @@ def test_launch_count_rule():
     assert bench.launches_per_step(W.WORKLOADS["skewed"], "auto") == 5
     assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=384), "auto") == 6
     assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=512), "auto") == 5
+    # bf16 weights take token tiles above 128 tokens, int8 weights above 256
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=128), "auto") == 3
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["prefill"], T=200), "auto") == 6
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["int8"], T=200), "auto") == 4
+    assert bench.launches_per_step(dataclasses.replace(W.WORKLOADS["int8"], T=300), "auto") == 4
     big = dataclasses.replace(W.WORKLOADS["prefill"], T=40000)   # > 1024 router blocks: + scan
     assert bench.launches_per_step(big, "auto") == 6
