@@ -342,9 +342,10 @@ def job_throughput(world, steps, work_per_step, t_max_ms):
 
 
 def weight_stream_form(wl, path):
-    """Whether the GEMMs run in the weight-stream orientation: forced, or on the
-    automatic path for small batches (T <= 256 with int8 weights, T <= 128 with
-    bf16 weights; the library's choice)."""
+    """Whether the step streams its weights (weight-stream down projection, a
+    bound set by HBM): forced, or on the automatic path for small batches
+    (T <= 256 with int8 weights, T <= 128 with bf16 weights, whose gate/up GEMM
+    then runs 128-row token tiles; the library's choice)."""
     if path == "weight_stream":
         return True
     if path != "auto":
@@ -566,7 +567,11 @@ def roofline_entry(wl, pk, stage_ms, touched, clocks, path="auto"):
         gu_bytes = touched * 2 * d * f * esz
         gu = gu_bytes / (gu_ms / 1e3) / 1e9
         dn = touched * d * f * esz / (dn_ms / 1e3) / 1e9
-        return {"bound": "hbm", "kernel": "moe_expert_gemm_kernel<GATEUP, WEIGHT_STREAM>",
+        # bf16 weights on the automatic path: the gate/up GEMM in 128-row token
+        # tiles, the down projection in weight-stream tiles
+        kern = ("moe_expert_gemm_kernel<GATEUP, TOKEN_TILE> (128-row tiles)"
+                if path == "auto" and wl.dtype == "bf16" else "moe_expert_gemm_kernel<GATEUP, WEIGHT_STREAM>")
+        return {"bound": "hbm", "kernel": kern,
                 "achieved": round(gu, 1), "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gu / pk["hbm_gbs"], 4),
                 "traffic": recorded_traffic(wl), "peak_source": f"{pk['source']} HBM copy",
                 "algorithmic_per_launch": gu_bytes,

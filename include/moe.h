@@ -100,7 +100,9 @@ typedef enum {
 /* Kernel family. AUTO picks WEIGHT_STREAM (tokens on the MMA N side, split-K
  * down projection) when the average tokens per expert is small (T <= 128 with
  * bf16 weights, T <= 256 with int8 weights; measured crossovers), else token
- * tiles (tokens on the MMA M side). With bf16 weights the gate/up
+ * tiles (tokens on the MMA M side). For those small bf16 batches only the down
+ * projection streams its weights that way; the gate/up GEMM runs 128-token
+ * tiles on single CTAs (measured faster). Above them, with bf16 weights the gate/up
  * GEMM then runs 256-token tiles on single CTAs from T = 512 on; below that,
  * and for the down GEMM, the device chooses from the expert counts between
  * 128-token tiles on single CTAs and 256-token tiles on CTA pairs

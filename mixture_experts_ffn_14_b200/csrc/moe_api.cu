@@ -225,7 +225,13 @@ WorkspaceLayout plan_workspace(int64_t T, int64_t d, int64_t f, moe_dtype_t dtyp
   const int64_t rows = 2 * T;
   L.nblk = (T + kRouteTokens - 1) / kRouteTokens;
   L.weight_stream = dtype != MOE_F32 && use_weight_stream(T, path, dtype);
-  L.tile_path = dtype != MOE_F32 && !L.weight_stream;
+  // Small bf16 batches on the automatic path: the gate/up GEMM in 128-row
+  // token tiles (interleaved runs at the Grok-1 shape, gate/up ms against
+  // weight-stream tiles: T = 16 0.880 / 0.897, T = 64 1.001-1.014 /
+  // 1.047-1.050, T = 128 1.012-1.030 / 1.053-1.057), the down projection in
+  // weight-stream tiles (T = 64 0.516-0.531 against 0.585-0.605 ms in token tiles).
+  L.gateup_tt = L.weight_stream && path == MOE_PATH_AUTO && dtype == MOE_BF16;
+  L.tile_path = dtype != MOE_F32 && (!L.weight_stream || L.gateup_tt);
   if (dtype == MOE_F32) {
     L.splits = 1;
   } else if (L.weight_stream) {
@@ -385,10 +391,10 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     g.splits = 1;
     g.act = o->activation;
     g.int8_weights = w8;
-    g.weight_stream = L.weight_stream;
+    g.weight_stream = L.weight_stream && !L.gateup_tt;
     // Small batches (<= 32 token slots per expert on average): weight-stream
     // tiles of at most 64 tokens, which leave room for more weight stages in flight.
-    g.short_tiles = L.weight_stream && T <= 128;
+    g.short_tiles = g.weight_stream && T <= 128;
     g.status = status;
     g.tile_counter = tile_counters;
     g.tile_counter_single = tile_counters + 2;
@@ -420,7 +426,13 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     // 1.21; T = 768 1.31 against 1.34-1.36; T = 4096 5.15-5.39 against
     // 5.67-5.80 before). The down projection keeps the choice above: its
     // epilogue, which 256-row tiles cannot overlap with the next tile, is heavier.
-    if (auto_tt && !gather_x && T >= kTallMinT) {
+    if (L.gateup_tt) {
+      // 128-row token tiles on single CTAs alone: with at most 32 rows per
+      // expert on average the CTA-pair form never pays.
+      TcGemmArgs gt = g;
+      gt.select = 0;
+      MOE_TRY(launch_tc_gateup(gt, stream));
+    } else if (auto_tt && !gather_x && T >= kTallMinT) {
       TcGemmArgs gt = g;
       gt.tall_tiles = true;
       gt.select = 0;
@@ -430,6 +442,8 @@ moe_status_t run_forward(const moe_args_t* a, const moe_options_t* o, const moe_
     }
     MOE_TRY(mark(3));
     TcGemmArgs g2 = g;
+    g2.weight_stream = L.weight_stream;
+    g2.short_tiles = L.weight_stream && T <= 128;
     g2.x = h;
     g2.row_token = nullptr;
     g2.w0 = a->w_down;
@@ -622,7 +636,8 @@ RouteLayout plan_route(int64_t T, int64_t d, moe_dtype_t dtype) {
 struct ExpertsLayout {
   size_t status, counts, offsets, ones, h, ypart, total;
   int32_t splits;
-  bool weight_stream;
+  bool weight_stream;  // down projection (and gate/up unless gateup_tt) in weight-stream tiles
+  bool gateup_tt;      // bf16, automatic path: gate/up in 128-row token tiles (as in the whole layer)
 };
 
 bool experts_sizes_ok(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype_t dtype) {
@@ -645,6 +660,7 @@ ExpertsLayout plan_experts(int64_t R, int64_t d, int64_t f, int32_t n, moe_dtype
   const int64_t ws_rows = dtype == MOE_BF16_INT8W ? 64 : 32;
   L.weight_stream = dtype != MOE_F32 && (path == MOE_PATH_WEIGHT_STREAM ||
                                          (path == MOE_PATH_AUTO && R <= ws_rows * static_cast<int64_t>(n)));
+  L.gateup_tt = L.weight_stream && path == MOE_PATH_AUTO && dtype == MOE_BF16;
   const int64_t kblocks = f / 64;
   if (down_splits > 0) {
     L.splits = kblocks % down_splits == 0 && dtype != MOE_F32 ? down_splits : (down_splits == 1 ? 1 : -1);
@@ -813,8 +829,8 @@ moe_status_t moe_experts_forward(const moe_expert_rows_t* a, const moe_options_t
   g.splits = 1;
   g.act = o->activation;
   g.int8_weights = w8;
-  g.weight_stream = L.weight_stream;
-  g.short_tiles = L.weight_stream && R <= 32 * static_cast<int64_t>(a->n_experts);
+  g.weight_stream = L.weight_stream && !L.gateup_tt;
+  g.short_tiles = g.weight_stream && R <= 32 * static_cast<int64_t>(a->n_experts);
   g.status = status;
   g.n_experts = a->n_experts;
   // One token-tile form per call here (the single-CTA one unless the pair form
@@ -827,6 +843,8 @@ moe_status_t moe_experts_forward(const moe_expert_rows_t* a, const moe_options_t
   };
   if (gemm(g, false) != cudaSuccess) return MOE_ERR_CUDA;
   TcGemmArgs g2 = g;
+  g2.weight_stream = L.weight_stream;
+  g2.short_tiles = L.weight_stream && R <= 32 * static_cast<int64_t>(a->n_experts);
   g2.x = h;
   g2.w0 = a->w_down;
   g2.w1 = nullptr;

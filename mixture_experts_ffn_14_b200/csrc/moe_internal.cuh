@@ -42,8 +42,11 @@ struct WorkspaceLayout {
   int64_t nblk;      // router / dispatch CTAs
   int32_t splits;    // split-K factor of the down projection
   int32_t router_slices;  // d slices of the router grid
-  bool weight_stream;
-  bool tile_path;    // token tiles (bf16 / int8 weights, not weight-stream): row gather possible
+  bool weight_stream;  // down projection in the weight-stream form (and gate/up unless gateup_tt)
+  // bf16 weights, automatic path, weight-stream batch: the gate/up GEMM runs
+  // 128-row token tiles on single CTAs, the down projection weight-stream tiles.
+  bool gateup_tt;
+  bool tile_path;    // gate/up in token tiles (bf16 / int8 weights): row gather possible
 };
 
 // Host: workspace layout for a call (valid arguments assumed).
