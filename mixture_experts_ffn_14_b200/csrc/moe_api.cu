@@ -171,13 +171,34 @@ bool use_weight_stream(int64_t T, moe_path_t path, moe_dtype_t dtype) {
   return T <= (dtype == MOE_BF16_INT8W ? 256 : 128);
 }
 
+// Expected row tiles of `rows` rows of one expert under balanced routing: a
+// token picks the expert with probability 1/4 (two of eight), so its count is
+// close to normal with mean m and variance 3m/4; E[ceil(count / rows)] is
+// summed over a grid of that density.
+double expected_row_tiles(double m, double rows) {
+  const double sd = std::sqrt(std::max(0.75 * m, 1e-9));
+  double tot = 0.0, wsum = 0.0;
+  for (int i = -40; i <= 40; ++i) {
+    const double z = i / 10.0, c = m + z * sd, w = std::exp(-0.5 * z * z);
+    if (c <= 0.0) continue;
+    tot += w * std::ceil(c / rows);
+    wsum += w;
+  }
+  return wsum > 0.0 ? tot / wsum : 0.0;
+}
+
 // Split-K factor of the token-tile down projection. Its tiles are long (K = f)
-// and few (rows/128 x d/256), so the last partial wave can idle most SMs. For
-// balanced loads (each expert pads on average half a tile) estimate, per split
-// factor s, the time of the waves of whichever tile form the kernels will pick
-// (single-CTA 128-row tiles, or CTA-pair 256-row tiles at a 7 % discount), plus
-// 2.3 % of the unsplit work per extra split for the fp32 partial sums that are
-// written and read again (their bytes relative to the GEMM time at d, f).
+// and few (rows/128 x d/256), so the last partial wave can idle most SMs. Per
+// split factor s, estimate the time of the waves of whichever tile form the
+// kernels will pick (single-CTA tiles, or CTA-pair 256-row tiles at a 7 %
+// discount) from the expected tile counts, plus 20 % of the unsplit work per
+// extra split. That cost is fitted to interleaved runs of forced split factors
+// (down ms, split 1 / 2 / 4): bf16 T = 160 0.644 / 0.565 / 0.572, T = 384
+// 0.677 / 0.608 / 0.632, T = 768 0.843 / 0.935 / 0.935, T = 2048 1.750 / 1.829
+// / 1.935; int8 T = 768 1.071 / 0.904 / 0.966, T = 1024 1.025 / 1.152 / 1.329,
+// T = 2048 1.965 / 1.972 / 2.118. The model picks the fastest factor at all
+// thirteen measured sizes; the earlier one (mean tiles + 0.5 per expert, 2.3 %
+// per split for the partial sums' bytes) was up to 16 % off.
 int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t requested, bool allow_single,
                                       bool allow_pair, int64_t single_rows) {
   const int64_t kblocks = f / 64;
@@ -185,8 +206,8 @@ int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t r
   auto valid = [&](int64_t s) { return s >= 1 && kblocks % s == 0 && kblocks / s >= 8; };
   const double per_expert = static_cast<double>(2 * T) / kE;
   const double nt = static_cast<double>(d / 256);
-  const double t1 = kE * (per_expert / single_rows + 0.5) * nt;  // expected single-CTA tiles
-  const double t2 = kE * (per_expert / 256.0 + 0.5) * nt;  // expected pair tiles
+  const double t1 = kE * expected_row_tiles(per_expert, static_cast<double>(single_rows)) * nt;  // single-CTA tiles
+  const double t2 = kE * expected_row_tiles(per_expert, 256.0) * nt;                                // pair tiles
   const double sms = device_sm_count(), pairs = sms / 2;
   int32_t best = 1;
   double best_t = 1e30;
@@ -195,7 +216,7 @@ int32_t choose_token_tile_down_splits(int64_t T, int64_t d, int64_t f, int32_t r
     double t = 1e30;
     if (allow_single) t = std::min(t, std::ceil(t1 * s / sms) / s);
     if (allow_pair) t = std::min(t, std::ceil(t2 * s / pairs) / s / 1.07);
-    t += 0.023 * (s - 1) * (t1 / sms);
+    t += 0.20 * (s - 1) * (t1 / sms);
     if (t < best_t - 1e-9) {
       best_t = t;
       best = static_cast<int32_t>(s);
