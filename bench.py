@@ -448,7 +448,7 @@ def main():
     int8 = skewed = None
     if wl.name == "prefill" and a.T is None and a.d is None and a.f is None:
         if not a.no_skewed:
-            # BASELINE's skewed-load config on the prefill weights: a fresh
+            # The skewed-load workload on the prefill weights: a fresh
             # T = 16384 batch and the per-expert router bias.
             ws = W.WORKLOADS["skewed"]
             inp_s = {k: inp[k] for k in ("w_router", "w_gate", "w_up", "w_down")}
@@ -762,7 +762,7 @@ def run_decode(a, moe, W, wl, inp, dev, pk):
 
 
 def run_side(a, moe, wl2, name, inp2, dev, pk, dist, world):
-    """One more BASELINE-shape workload measured like the main line: K timed
+    """One more Grok-1-shape workload measured like the main line: K timed
     steps with an L2 flush between them, CUDA events on the launching stream,
     the library's stage events, clocks sampled during the steps, its own
     roofline entry and a bounded oracle sample on the host cores."""

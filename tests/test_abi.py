@@ -67,6 +67,27 @@ def test_workspace_size_rules():
         assert N.lib().moe_workspace_size(T, d, f, 8, 2, dt) == N.lib().moe_workspace_size_ex(T, d, f, 8, 2, dt, 0, 0)
 
 
+def test_form_and_split_choices_at_the_grok_shape():
+    # Seen through the workspace size (weight-stream layouts keep four combine
+    # counters per token and column tile, and every split its own fp32 partial
+    # sums). Weight-stream form up to 128 tokens with bf16 weights, up to 256
+    # with int8 weights; token tiles above.
+    d, f = 6144, 32768
+
+    def ws(T, dt, path=moe.MOE_PATH_AUTO, splits=0):
+        return moe.moe_workspace_size(T, d, f, dtype=dt, path=path, down_splits=splits)
+
+    for dt, last in ((moe.MOE_BF16, 128), (moe.MOE_BF16_INT8W, 256)):
+        assert ws(last, dt) == ws(last, dt, moe.MOE_PATH_WEIGHT_STREAM)
+        assert ws(last + 1, dt) != ws(last + 1, dt, moe.MOE_PATH_WEIGHT_STREAM)
+    # the token-tile down projection's split factor (a measured model): two
+    # splits for a few rows per expert, none once the tiles fill the SMs
+    for dt, T, want in ((moe.MOE_BF16, 384, 2), (moe.MOE_BF16, 768, 1), (moe.MOE_BF16, 4096, 1),
+                        (moe.MOE_BF16_INT8W, 768, 2), (moe.MOE_BF16_INT8W, 1024, 1)):
+        got = [s for s in (1, 2, 4, 8) if ws(T, dt, splits=s) == ws(T, dt)]
+        assert got == [want], (dt, T, got)
+
+
 def _args(T=64, d=512, f=384, E=8, k=2, dtype=moe.MOE_BF16, base=0x10000000):
     # Fake, never dereferenced device addresses: every call below must return
     # from the host-side checks before any CUDA call.
